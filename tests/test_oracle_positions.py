@@ -1,0 +1,212 @@
+"""Pins for the oracle's position planes (CPU only).
+
+Each test ties the oracle to something other than itself: the pages' worked
+values (golden files), the structure of the 8x8 grid, the text-only special
+case, the red arms that the pages report as failing, and a brute-force
+comparison with a segment-by-segment construction of the canvas.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.helpers import golden_rows
+from vlm_decoder_positional_b200 import inputs
+
+MARK = inputs.IMAGE_TOKEN_ID
+TEXT_ONLY_START = 2 ** 30
+
+
+def one_prompt(length, origin, seed=7, row_ids="v_plus_k"):
+    rng = np.random.default_rng(seed)
+    ids = inputs.prompt_ids(rng, length, origin, row_ids)
+    return ids, np.array([0, length], dtype=np.int32)
+
+
+def test_golden_o6_table_matches_config_1():
+    wl = inputs.make_config(1, with_qk=False)
+    pos, start, amount = oracle.positions(wl.ids, wl.cu_seqlens, MARK)
+    want = np.array([[int(v) for v in r] for r in golden_rows("canvas_O6_80.txt")])
+    assert want.shape == (80, 4) and (want[:, 0] == np.arange(80)).all()
+    np.testing.assert_array_equal(pos.T, want[:, 1:])
+    assert (int(start[0]), int(amount[0])) == (73, 58)
+
+
+@pytest.mark.parametrize("row", golden_rows("shift_worked.txt"))
+def test_worked_shift_values(row):
+    O, want_start, want_amount, first_after = (int(v) for v in row)
+    ids, cu = one_prompt(O + 120, O)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    assert int(start[0]) == want_start and int(amount[0]) == want_amount
+    assert pos[:, want_start].tolist() == [first_after] * 3
+    # the first text token after the frame sits at O + 9 (9 = max(H, W) + 1)
+    assert first_after == O + 9
+
+
+@pytest.mark.parametrize("O", [0, 1, 6, 17, 40, 3000])
+def test_rows_tile_the_8x8_grid_row_major(O):
+    ids, cu = one_prompt(O + 80, O)
+    pos, _, _ = oracle.positions(ids, cu, MARK)
+    rows = pos[:, O + 1:O + 65]
+    assert (rows[0] == O).all()
+    cells = list(zip((rows[1] - O).tolist(), (rows[2] - O).tolist()))
+    assert cells == [(r, c) for r in range(8) for c in range(8)]
+
+
+@pytest.mark.parametrize("O", [0, 5, 33])
+def test_frame_ranges_and_monotone_tail(O):
+    n = O + 300
+    ids, cu = one_prompt(n, O)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    frame = pos[:, O:O + 67]
+    assert (frame[0] == O).all()
+    assert frame[1:].min() == O - 1 and frame[1:].max() == O + 8
+    tail = pos[:, int(start[0]):]
+    assert (tail[0] == tail[1]).all() and (tail[1] == tail[2]).all()
+    assert (np.diff(tail[0]) == 1).all()
+    assert (pos[0] <= np.arange(n)).all()
+
+
+def test_text_only_is_one_dimensional():
+    ids, cu = one_prompt(500, -1)
+    assert not (ids == MARK).any()
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    assert int(start[0]) == TEXT_ONLY_START and int(amount[0]) == 0
+    for r in range(3):
+        np.testing.assert_array_equal(pos[r], np.arange(500))
+
+
+def canvas_by_segments(ids, marker):
+    """Independent construction: text advances a running counter on all three
+    planes; the first <image> lays the 67-token frame on a canvas anchored at
+    the counter; text after the frame resumes one past the largest coordinate
+    the canvas used (the pages' 9 = max(H, W) + 1)."""
+    out, nxt, i, seen = [], 0, 0, False
+    n = len(ids)
+    while i < n:
+        if ids[i] == marker and not seen:
+            seen = True
+            o = nxt
+            frame = ([(o, o - 1, o - 1)]
+                     + [(o, o + r, o + c) for r in range(8) for c in range(8)]
+                     + [(o, o + 8, o + 8), (o, o, o)])
+            take = min(len(frame), n - i)
+            out += frame[:take]
+            i += take
+            nxt = max(max(v) for v in frame) + 1
+        else:
+            out.append((nxt, nxt, nxt))
+            nxt += 1
+            i += 1
+    return np.array(out, dtype=np.int64).T.reshape(3, n)
+
+
+def test_brute_force_every_origin_and_position():
+    rng = np.random.default_rng(3)
+    prompts, origins = [], list(range(0, 101))
+    for O in origins:
+        prompts.append(inputs.prompt_ids(rng, 201, O))
+    ids, cu = inputs.pack(prompts)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    for b, O in enumerate(origins):
+        seg = ids[cu[b]:cu[b + 1]]
+        want = canvas_by_segments(seg.tolist(), MARK)
+        np.testing.assert_array_equal(pos[:, cu[b]:cu[b + 1]], want, err_msg=f"O={O}")
+        assert (int(start[b]), int(amount[b])) == (O + 67, 58)
+
+
+def test_first_marker_wins_and_later_markers_are_text():
+    ids, cu = one_prompt(400, 10)
+    ids[200] = MARK
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    assert int(start[0]) == 77
+    assert pos[:, 200].tolist() == [200 - 58] * 3
+    want = canvas_by_segments(ids.tolist(), MARK)
+    np.testing.assert_array_equal(pos, want)
+
+
+def test_truncated_frame_and_origin_zero():
+    ids, cu = one_prompt(40, 0)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    assert pos[:, 0].tolist() == [0, -1, -1]
+    assert (int(start[0]), int(amount[0])) == (67, 58)
+    np.testing.assert_array_equal(pos, canvas_by_segments(ids.tolist(), MARK))
+
+
+def test_pad_row_ids_give_the_same_planes():
+    a, cu = one_prompt(150, 12, row_ids="v_plus_k")
+    b, _ = one_prompt(150, 12, row_ids="pad")
+    assert (a != b).any()
+    np.testing.assert_array_equal(oracle.positions(a, cu, MARK)[0],
+                                  oracle.positions(b, cu, MARK)[0])
+
+
+def test_packed_batch_with_empty_sequences_is_per_sequence():
+    rng = np.random.default_rng(11)
+    lens, origins = [0, 90, 0, 130, 1, 70], [-1, 3, -1, -1, -1, 0]
+    prompts = [inputs.prompt_ids(rng, n, o) for n, o in zip(lens, origins)]
+    ids, cu = inputs.pack(prompts)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    for b, p in enumerate(prompts):
+        pb, sb, ab = oracle.positions(p, np.array([0, len(p)], np.int32), MARK)
+        np.testing.assert_array_equal(pos[:, cu[b]:cu[b + 1]], pb)
+        assert (start[b], amount[b]) == (sb[0], ab[0])
+
+
+def test_malformed_cu_seqlens_rejected():
+    ids = np.zeros(10, np.int32)
+    for cu in ([0, 5, 4, 10], [1, 10], [0, 9]):
+        with pytest.raises(oracle.OracleError):
+            oracle.positions(ids, np.array(cu, np.int32), MARK)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_red_arms_fail_on_every_image_prompt(cfg):
+    # The pages' negative controls: "amount + 1" and "1-D planes" must give
+    # different planes; on text-only prompts every arm agrees.
+    wl = inputs.make_config(cfg, with_qk=False)
+    green = oracle.positions(wl.ids, wl.cu_seqlens, MARK)[0]
+    plus1 = oracle.positions(wl.ids, wl.cu_seqlens, MARK, rule="amount+1")[0]
+    flat = oracle.positions(wl.ids, wl.cu_seqlens, MARK, rule="planes_1d")[0]
+    cu = wl.cu_seqlens
+    for b in range(wl.num_seqs):
+        s = slice(cu[b], cu[b + 1])
+        O = int(wl.frame_origin[b])
+        if O < 0:
+            assert (green[:, s] == plus1[:, s]).all() and (green[:, s] == flat[:, s]).all()
+            continue
+        assert (green[:, s] != flat[:, s]).any()
+        assert (green[:, s] != plus1[:, s]).any()
+        # only the text before the frame still matches under amount + 1: the
+        # graph derives the origin from (start, amount), so the frame moves too
+        pre = slice(cu[b], cu[b] + max(O - 1, 0))
+        assert (green[:, pre] == plus1[:, pre]).all()
+        rest = slice(cu[b] + max(O - 1, 0), cu[b + 1])
+        assert (green[:, rest] != plus1[:, rest]).any(axis=0).all()
+
+
+def test_step_form_reproduces_the_prompt_planes():
+    # cmr_positions_step receives only (p, start, amount); it must give the
+    # same planes as the prompt rule at every index of an image prompt and of
+    # a text-only prompt, and p - amount for every token after the frame.
+    rng = np.random.default_rng(5)
+    prompts = [inputs.prompt_ids(rng, 300, 6), inputs.prompt_ids(rng, 300, 17),
+               inputs.prompt_ids(rng, 300, -1), inputs.prompt_ids(rng, 300, 0)]
+    ids, cu = inputs.pack(prompts)
+    pos, start, amount = oracle.positions(ids, cu, MARK)
+    for b in range(len(prompts)):
+        n = 300
+        p = np.arange(n, dtype=np.int32)
+        step = oracle.positions_step(p, np.full(n, start[b]), np.full(n, amount[b]))
+        np.testing.assert_array_equal(step, pos[:, cu[b]:cu[b + 1]])
+    # generated tokens (p beyond the prompt) sit at p - 58 on all three planes
+    gen = np.arange(300, 400, dtype=np.int32)
+    step = oracle.positions_step(gen, np.full(100, start[0]), np.full(100, amount[0]))
+    assert (step == gen - 58).all()
+
+
+def test_decode_config_positions():
+    wl = inputs.make_config(4, with_qk=False)
+    _, start, amount = oracle.positions(wl.ids, wl.cu_seqlens, MARK)
+    assert (amount == 58).all() and (start == wl.frame_origin + 67).all()
+    step = oracle.positions_step(wl.cache_len, start, amount)
+    assert (step == wl.cache_len - 58).all()
