@@ -1,0 +1,426 @@
+"""Benchmark of the canvas M-RoPE hot path on B200.
+
+One step = the whole path over one batch: cmr_positions (planes from ids) then
+cmr_rotate_qk (fused cos/sin + rotate of Q and K, every layer), on the
+6-layer workload: 32 prompts x 8192 tokens with one image frame each, Q [6,
+262144, 8, 256] and K [6, 262144, 2, 256] bf16, rot_dim 64, theta 1e7,
+sections [11, 11, 10].  The rotate kernel touches 4.03 GB per step, far more
+than the 126 MB L2, so no L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (weak scaling: one batch per GPU)
+
+Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle
+(single thread) on a bounded sample of the same workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vlm_decoder_positional_b200 import cmr, inputs  # noqa: E402
+
+METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/K, 1 GPU"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
+                  "vlm_decoder_positional_b200/csrc/cmr_internal.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_qk_traffic.txt")
+
+# Algorithmic bytes: rotate reads and writes the rot_dim dims of every Q and K
+# head of every layer (2,560 B per token-layer here) and reads pos once (12 B
+# per token); positions reads 4 B of ids and writes 12 B of planes per token.
+def rotate_bytes(n_tokens, layers, hq, hk, rot_dim):
+    return n_tokens * layers * (hq + hk) * rot_dim * 2 * 2 + n_tokens * 12
+
+
+def positions_bytes(n_tokens, num_seqs):
+    return n_tokens * 16 + num_seqs * 12
+
+
+def workload_label(wl):
+    t = wl.num_seqs if wl.cache_len is not None else wl.n_tokens  # Q/K tokens of the workload
+    return (f"{wl.name}: {wl.num_seqs} prompts x {wl.n_tokens // max(wl.num_seqs, 1)} tokens, "
+            f"{wl.num_layers} layers, Q [{wl.num_layers},{t},{wl.hq},{wl.head_dim}] "
+            f"K [{wl.num_layers},{t},{wl.hk},{wl.head_dim}] bf16, rot_dim "
+            f"{wl.rot_dim}, theta {wl.theta:g}, sections {list(wl.sections)}")
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def rotate_source_hash():
+    h = hashlib.sha256()
+    for rel in ROTATE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    this exact kernel source and workload; otherwise None."""
+    try:
+        rec = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.strip()
+        if rec.get("kernel_source_sha256") != rotate_source_hash():
+            return None
+        if rec.get("workload") != workload_name:
+            return None
+        return int(rec["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, interval=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self._nvml = None
+            self.error = str(e)
+
+    def _sample(self):
+        n = self._nvml
+        self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+        mask = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        for name, bit in self.REASONS.items():
+            if mask & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self._nvml:
+            self._sample()
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+            self._sample()
+
+    def summary(self):
+        if not self._nvml:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.error}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "nvml"}
+
+
+# ---------------------------------------------------------------------------
+# CPU side: the oracle on a bounded sample (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(wl_cpu, n_seqs, n_tokens):
+    """One oracle pass over a sample: planes of the first n_seqs prompts, then
+    the rotation of their first n_tokens tokens, every layer and head."""
+    import oracle
+    cu = wl_cpu["cu"][: n_seqs + 1]
+    ids = wl_cpu["ids"][: cu[-1]]
+    pos, _, _ = oracle.positions(ids, cu, inputs.IMAGE_TOKEN_ID)
+    p = np.ascontiguousarray(pos[:, :n_tokens])
+    oracle.rotate_bf16(wl_cpu["q"][:, :n_tokens], p)
+    oracle.rotate_bf16(wl_cpu["k"][:, :n_tokens], p)
+    return n_tokens
+
+
+def cpu_sample_inputs(wl, n_tokens):
+    def bits(t):
+        return t[:, :n_tokens].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return {"ids": wl.ids, "cu": wl.cu_seqlens, "q": bits(wl.q), "k": bits(wl.k)}
+
+
+def calibrate_sample(wl_cpu, seconds):
+    probe = 64
+    t0 = time.perf_counter()
+    oracle_sample_step(wl_cpu, 1, probe)
+    dt = time.perf_counter() - t0
+    return int(max(probe, min(wl_cpu["q"].shape[1], probe * seconds / max(dt, 1e-6))))
+
+
+def run_cpu_baseline(wl, seconds):
+    cap = 8192
+    wl_cpu = cpu_sample_inputs(wl, cap)
+    n = calibrate_sample(wl_cpu, seconds)
+    n = min(n, cap)
+    t0 = time.perf_counter()
+    oracle_sample_step(wl_cpu, 1, n)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"planes of prompt 0 ({wl.cu_seqlens[1]} tokens) + rotation of its first "
+                      f"{n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, "
+                      f"1 thread, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    # the same prompts (ids); Q/K drawn only for the sampled first prompt
+    wl = inputs.make_config(args.workload, device="cpu", with_qk=False)
+    first = int(wl.cu_seqlens[1]) if wl.cache_len is None else wl.num_seqs
+    wl.q = inputs.random_qk((wl.num_layers, min(first, 8192), wl.hq, wl.head_dim), wl.seed + 1)
+    wl.k = inputs.random_qk((wl.num_layers, min(first, 8192), wl.hk, wl.head_dim), wl.seed + 2)
+    per_step = max(1.0, args.reference_budget_s / (args.steps + args.warmup))
+    wl_cpu = cpu_sample_inputs(wl, 8192)
+    n = min(calibrate_sample(wl_cpu, per_step), 8192)
+    for _ in range(args.warmup):
+        oracle_sample_step(wl_cpu, 1, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(wl_cpu, 1, n)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"per step: planes of prompt 0 ({wl.cu_seqlens[1]} tokens) + rotation of its "
+              f"first {n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": workload_label(wl), "global_batch": wl.n_tokens,
+                   "seq_len": wl.n_tokens // wl.num_seqs, "parallelism": "cpu oracle, 1 thread"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU side
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    cmr.lib()
+
+    # weak scaling: every rank rotates its own batch (a different seed per rank)
+    wl = inputs.make_config(args.workload, device=dev,
+                            seed=inputs.BASE_SEED + args.workload + 1000 * rank)
+    ids = torch.from_numpy(wl.ids).to(dev)
+    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+    n, b, L = wl.n_tokens, wl.num_seqs, wl.num_layers
+    pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+    start = torch.empty(b, dtype=torch.int32, device=dev)
+    amount = torch.empty(b, dtype=torch.int32, device=dev)
+    decode = wl.cache_len is not None
+    cache_len = torch.from_numpy(wl.cache_len).to(dev) if decode else None
+    pos_step = torch.empty((3, b), dtype=torch.int32, device=dev) if decode else None
+    stream = torch.cuda.current_stream(dev)
+    tokens_per_step = wl.qk_tokens
+    rot_b = rotate_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim)
+
+    def step(ev=None):
+        p, s, a = cmr.positions(ids, cu, wl.image_token_id, out=(pos, start, amount))
+        pr = cmr.positions_step(cache_len, s, a, out=pos_step) if decode else p
+        if ev is not None:
+            ev[0].record(stream)
+        cmr.rotate_qk(wl.q, wl.k, pr, wl.theta, wl.sections, wl.rot_dim)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    rot_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        t_begin.record(stream)
+        for i in range(args.steps):
+            step(rot_events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    ms = t_begin.elapsed_time(t_end)
+    rot_ms = [a.elapsed_time(z) for a, z in rot_events]
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    launches = args.steps * (3 if decode else 2)
+
+    # end to end through the public API from pinned host memory
+    e2e = run_e2e(args, wl, dev, stream, dist)
+
+    if rank == 0:
+        peak, peak_src = measured_peak()
+        rot_avg_s = statistics.mean(rot_ms) / 1e3
+        achieved = rot_b / rot_avg_s / 1e9
+        traffic = recorded_traffic(wl.name)
+        value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = run_cpu_baseline(wl, args.cpu_seconds)
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K, uniform text ids, one 448x448 frame "
+                    "per prompt)",
+            "config": {"workload": workload_label(wl), "global_batch": n * world,
+                       "seq_len": n // max(b, 1), "parallelism": f"dp{world} (independent "
+                       "batches, no data-path collective)",
+                       "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
+                             " no flush" % (rot_b / 1e9)},
+            "hbm_gbs": achieved, "pct_of_peak": 100.0 * achieved / peak,
+            "token_layers_per_s": value * L,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "rotate_qk_kernel",
+                         "algorithmic_bytes_per_launch": rot_b,
+                         "avg_launch_ms": rot_avg_s * 1e3,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_src == "measured" else "fallback 6650 GB/s"},
+            "positions_bytes_per_step": positions_bytes(n, b),
+            "e2e": e2e, "gpu_launches": launches, "clocks": clocks.summary(),
+            "cpu_baseline": cpu, "impl": "ours",
+        }
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, wl, dev, stream, dist):
+    """Same metric through the public API: every step copies the inputs from
+    pinned host memory, runs positions + rotate, and reads the results back."""
+    steps = max(2, min(args.steps, args.e2e_steps))
+    h_ids = torch.from_numpy(wl.ids).pin_memory()
+    h_cu = torch.from_numpy(wl.cu_seqlens).pin_memory()
+    h_q = torch.empty(wl.q.shape, dtype=wl.q.dtype, pin_memory=True)
+    h_k = torch.empty(wl.k.shape, dtype=wl.k.dtype, pin_memory=True)
+    h_q.copy_(wl.q)
+    h_k.copy_(wl.k)
+    decode = wl.cache_len is not None
+    h_cl = torch.from_numpy(wl.cache_len).pin_memory() if decode else None
+    npos = wl.qk_tokens
+    h_pos = torch.empty((3, npos), dtype=torch.int32, pin_memory=True)
+    h_start = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
+    h_amount = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
+
+    def step():
+        ids = h_ids.to(dev, non_blocking=True)
+        cu = h_cu.to(dev, non_blocking=True)
+        q = h_q.to(dev, non_blocking=True)
+        k = h_k.to(dev, non_blocking=True)
+        pos, start, amount = cmr.positions(ids, cu, wl.image_token_id)
+        if decode:
+            pos = cmr.positions_step(h_cl.to(dev, non_blocking=True), start, amount)
+        cmr.rotate_qk(q, k, pos, wl.theta, wl.sections, wl.rot_dim)
+        h_q.copy_(q, non_blocking=True)
+        h_k.copy_(k, non_blocking=True)
+        h_pos.copy_(pos, non_blocking=True)
+        h_start.copy_(start, non_blocking=True)
+        h_amount.copy_(amount, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    z.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = torch.tensor([a.elapsed_time(z)], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    world = dist.get_world_size() if dist else 1
+    h2d = (h_ids.numel() * 4 + h_cu.numel() * 4 + h_q.numel() * 2 + h_k.numel() * 2
+           + (h_cl.numel() * 4 if decode else 0))
+    d2h = h_q.numel() * 2 + h_k.numel() * 2 + h_pos.numel() * 4 + 8 * wl.num_seqs
+    return {"value": wl.qk_tokens * steps * world / (float(ms.item()) / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": float(ms.item()) / steps,
+            "path": "pinned host -> cmr.positions + cmr.rotate_qk -> pinned host"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=5, choices=[1, 2, 3, 4, 5],
+                    help="1..5: single 80-token prompt, varlen 16, 64x4096 outliers, "
+                         "decode 1024, 6 layers x 32 x 8192 (default)")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-budget-s", type=float, default=150.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

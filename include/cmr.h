@@ -1,0 +1,155 @@
+/*
+ * cmr.h -- canvas M-RoPE for the Qwen3.5-hybrid decoder of MiniCPM-V-4.7-1B,
+ * as a C ABI over hand-written sm_100a (B200) CUDA kernels.
+ *
+ * Two steps (HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides
+ * the text-only engine"; Core AI model zoo port notes, "The canvas rule and
+ * why the gate is on the planes"):
+ *   1. positions: the three position planes (T, H, W) of every token, derived
+ *      from the token ids by the canvas rule;
+ *   2. rotate: rotate-half M-RoPE of the Q and K heads of the full-attention
+ *      layers, in place, with cos/sin built per frequency from the plane that
+ *      the interleaved sections (e.g. [11, 11, 10]) assign to it.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named "device" must point to memory the current CUDA device can
+ *     read/write (cudaMalloc, torch CUDA tensors, managed memory).  Host
+ *     pointers are rejected with CMR_EINVAL where the runtime can tell.
+ *   - The caller owns every buffer.  The library never allocates, frees or
+ *     synchronises; all work is enqueued on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and runs asynchronously.
+ *   - Arguments are validated on the host before anything is enqueued; on any
+ *     non-CMR_OK return nothing was enqueued, except CMR_ECUDA from a launch,
+ *     which means the launch itself failed.  cmr_last_error_message() then
+ *     gives a one-line reason (per calling thread).
+ *   - Kernels never trap.  Malformed device-side data (cu_seqlens) is reported
+ *     through an optional device status word.
+ */
+#ifndef CMR_H_
+#define CMR_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CMR_API __attribute__((visibility("default")))
+#else
+#define CMR_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* cmr_stream_t;
+
+typedef enum cmr_status {
+  CMR_OK = 0,
+  CMR_EINVAL = 1,       /* an argument is out of range, misaligned or null */
+  CMR_ECUDA = 2,        /* a CUDA runtime call or a kernel launch failed */
+  CMR_EUNSUPPORTED = 3  /* valid, but outside the shapes this build handles */
+} cmr_status;
+
+/* Bits a kernel ORs into the optional device status word. */
+#define CMR_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens not 0 .. n_tokens, non-decreasing */
+
+/* Planes of a packed batch of prompts (the canvas table, HF card
+ * mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides the text-only
+ * engine").  For prompt b, O = the first local index whose id equals
+ * image_token_id (the <image> marker, 248078 for this model).  Then, for each
+ * local index p:
+ *   p <  O                 -> (p, p, p)
+ *   p == O                 -> (O, O-1, O-1)
+ *   p == O + 1 + k, k < 64 -> (O, O + k/8, O + k%8)   (8x8 grid, row-major)
+ *   p == O + 65            -> (O, O+8, O+8)
+ *   O + 65 < p < start     -> (O, O, O)
+ *   p >= start             -> (p - amount) on all three planes
+ * with start = O + 67 and amount = start - (O + 9) = 58 (port notes: "start =
+ * i0 + 67", "amount = 58").  A prompt with no marker is text-only: start =
+ * 2^30, amount = 0, every token (p, p, p).  Later markers in a prompt are
+ * ordinary tokens.  Frames cut off by the end of a prompt keep the rows that
+ * exist; start still reads O + 67.
+ *
+ *   ids          device int32 [n_tokens], prompts packed back to back
+ *   cu_seqlens   device int32 [num_seqs + 1]: cu[0] = 0, non-decreasing,
+ *                cu[num_seqs] = n_tokens; prompt b is ids[cu[b] .. cu[b+1])
+ *   num_seqs     >= 0 (0 requires n_tokens == 0)
+ *   n_tokens     0 .. INT32_MAX
+ *   out_pos      device int32 [3, n_tokens], plane-major: T row, H row, W row
+ *   out_start, out_amount   device int32 [num_seqs]
+ *   device_status  optional device int32 [1] (may be NULL).  If cu_seqlens is
+ *                malformed, the kernel ORs CMR_DEVICE_BAD_CU_SEQLENS into it
+ *                and writes nothing for the prompts whose bounds are invalid.
+ *                The library never clears it.
+ * Errors: CMR_EINVAL for null required pointers, negative sizes, num_seqs = 0
+ * with n_tokens > 0, or n_tokens > INT32_MAX. */
+CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
+                         int32_t num_seqs, int64_t n_tokens,
+                         int32_t image_token_id, int32_t* out_pos,
+                         int32_t* out_start, int32_t* out_amount,
+                         int32_t* device_status, cmr_stream_t stream);
+
+/* Planes of one new token per sequence, for decode and continuation (port
+ * notes: "every generated token at p - amount"; canvas table row "everything
+ * after the frame, generated tokens included").  Token b sits at absolute
+ * index p = cache_len[b] of its sequence, whose start / amount came from
+ * cmr_positions.  As in the engine, which binds only start and amount, the
+ * origin follows from amount = start - (O + 9); the token then gets the row of
+ * the canvas table above for index p (p >= start -> (p - amount) x 3; the
+ * text-only pair (2^30, 0) gives (p, p, p)).
+ *
+ *   cache_len, start, amount   device int32 [num_seqs]
+ *   out_pos      device int32 [3, num_seqs], plane-major
+ * Errors: CMR_EINVAL for null pointers or num_seqs < 0. */
+CMR_API cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* start,
+                              const int32_t* amount, int32_t num_seqs,
+                              int32_t* out_pos, cmr_stream_t stream);
+
+/* Rotate Q and K in place with interleaved M-RoPE (HF card "What it is":
+ * three planes T, H, W with interleaved sections [11, 11, 10]; port notes:
+ * `_mrope_freq_masks`, `forward_stateful_core(cos_sin=...)`).
+ * With F = rot_dim / 2 frequencies, frequency j belongs to plane
+ *   H if j % 3 == 1 and j < 3 * sections[1],
+ *   W if j % 3 == 2 and j < 3 * sections[2],
+ *   T otherwise,
+ * has inv_freq_j = theta^(-2j / rot_dim), and at token t turns the pair
+ * (x_j, x_{j+F}) of every head by a = pos[plane_j][t] * inv_freq_j:
+ *   x_j     <- x_j cos a - x_{j+F} sin a
+ *   x_{j+F} <- x_{j+F} cos a + x_j sin a
+ * Dims rot_dim .. head_dim-1 are not read or written.  The angle is formed and
+ * reduced modulo 2*pi in fp64, cos/sin and the rotation run in fp32, and the
+ * result is rounded to bf16 (nearest-even).
+ *
+ *   q      device bf16 [num_layers, n_tokens, hq, head_dim], 16-byte aligned
+ *   k      device bf16 [num_layers, n_tokens, hk, head_dim], 16-byte aligned
+ *          (either may be NULL when its head count is 0)
+ *   pos    device int32 [3, n_tokens] (plane-major), shared by every layer
+ *   n_tokens >= 0, num_layers >= 0 (either 0: nothing to do, CMR_OK)
+ *   hq, hk >= 0 with hq + hk >= 1
+ *   head_dim  multiple of 8
+ *   theta  > 0 and finite (1e7 for this model)
+ *   sections  host int32 [3] = {T, H, W} frequency counts, summing to
+ *          rot_dim / 2, each realisable by the interleave above
+ *   rot_dim   multiple of 16, 16 .. min(head_dim, 256)  (64 for this model)
+ * Errors: CMR_EINVAL for any violation above; CMR_EUNSUPPORTED when
+ * (hq + hk) * rot_dim / 16 > 512. */
+CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
+                         int32_t num_layers, int32_t hq, int32_t hk,
+                         int32_t head_dim, double theta,
+                         const int32_t sections[3], int32_t rot_dim,
+                         cmr_stream_t stream);
+
+/* Static, never-null description of a status code. */
+CMR_API const char* cmr_status_string(cmr_status s);
+
+/* One-line reason for the last non-CMR_OK return on the calling thread. */
+CMR_API const char* cmr_last_error_message(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+CMR_API int32_t cmr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CMR_H_ */

@@ -1,0 +1,98 @@
+"""The C-ABI library loads and exports every entry point include/cmr.h
+declares, and rejects bad arguments on the host before touching a GPU.
+No call here reaches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from vlm_decoder_positional_b200 import build as libbuild
+from vlm_decoder_positional_b200 import cmr
+
+HEADER = os.path.join(libbuild.INCLUDE, "cmr.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    return cmr.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"CMR_API\s+[\w\s\*]+?\b(cmr_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert set(names) == {"cmr_positions", "cmr_positions_step", "cmr_rotate_qk",
+                          "cmr_status_string", "cmr_last_error_message", "cmr_version"}
+    assert set(names) == set(cmr.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", libbuild.LIB], check=True,
+                         capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+    ours = {s for s in exported if s.startswith("cmr") or "cmr" in s.lower()}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings_and_version(lib):
+    for code in (0, 1, 2, 3):
+        assert lib.cmr_status_string(code)
+    assert b"unknown" in lib.cmr_status_string(99)
+    assert lib.cmr_version() == 10000
+
+
+SEC = (ctypes.c_int32 * 3)(11, 11, 10)
+FAKE = 0x10000  # a 16-byte aligned address; never dereferenced
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n_tokens=-1), dict(num_layers=-1), dict(hq=0, hk=0), dict(hq=-1),
+    dict(head_dim=250), dict(rot_dim=24), dict(rot_dim=0), dict(rot_dim=512, head_dim=512),
+    dict(rot_dim=128, head_dim=64), dict(theta=0.0), dict(theta=float("inf")),
+    dict(theta=float("nan")), dict(sections=(12, 11, 10)), dict(sections=(0, 20, 12)),
+    dict(q=FAKE + 2), dict(k=FAKE + 8), dict(q=None), dict(pos=None), dict(sections=None),
+])
+def test_rotate_rejects_bad_arguments_on_the_host(lib, kw):
+    a = dict(q=FAKE, k=FAKE, pos=FAKE, n_tokens=10, num_layers=1, hq=8, hk=2, head_dim=256,
+             theta=1e7, sections=(11, 11, 10), rot_dim=64)
+    a.update(kw)
+    sec = None if a["sections"] is None else (ctypes.c_int32 * 3)(*a["sections"])
+    st = lib.cmr_rotate_qk(a["q"], a["k"], a["pos"], a["n_tokens"], a["num_layers"], a["hq"],
+                           a["hk"], a["head_dim"], a["theta"], sec, a["rot_dim"], None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+    assert lib.cmr_last_error_message()
+
+
+def test_rotate_too_many_heads_is_unsupported(lib):
+    st = lib.cmr_rotate_qk(FAKE, FAKE, FAKE, 10, 1, 100, 29, 256, 1e7, SEC, 64, None)
+    assert st == cmr.CMR_EUNSUPPORTED
+
+
+def test_rotate_empty_work_is_a_no_op(lib):
+    assert lib.cmr_rotate_qk(None, None, None, 0, 1, 8, 2, 256, 1e7, SEC, 64, None) == 0
+    assert lib.cmr_rotate_qk(None, None, None, 10, 0, 8, 2, 256, 1e7, SEC, 64, None) == 0
+
+
+@pytest.mark.parametrize("args", [
+    (FAKE, FAKE, -1, 10), (FAKE, FAKE, 1, -1), (FAKE, FAKE, 0, 10), (FAKE, FAKE, 1, 2 ** 31),
+    (FAKE, None, 1, 10), (None, FAKE, 1, 10),
+])
+def test_positions_rejects_bad_arguments_on_the_host(lib, args):
+    ids, cu, b, n = args
+    st = lib.cmr_positions(ids, cu, b, n, 248078, FAKE if ids else None, FAKE, FAKE, None, None)
+    assert st == cmr.CMR_EINVAL
+
+
+def test_positions_empty_batch_is_a_no_op(lib):
+    assert lib.cmr_positions(None, None, 0, 0, 248078, None, None, None, None, None) == 0
+    assert lib.cmr_positions_step(None, None, None, 0, None, None) == 0
+    assert lib.cmr_positions_step(None, None, None, -1, None, None) == cmr.CMR_EINVAL

@@ -1,1 +1,13 @@
-"""Canvas M-RoPE for the Qwen3.5-hybrid decoder of MiniCPM-V-4.7-1B, on B200."""
+"""Canvas M-RoPE for the Qwen3.5-hybrid decoder of MiniCPM-V-4.7-1B, on B200.
+
+    pos, start, amount = positions(ids, cu_seqlens)        # planes (T, H, W)
+    rotate_qk(q, k, pos, theta=1e7, sections=(11, 11, 10), rot_dim=64)
+
+Both run hand-written sm_100a kernels in libcmr.so through its C ABI
+(include/cmr.h); build it with ``python -m vlm_decoder_positional_b200.build``.
+"""
+from .cmr import (CMR_DEVICE_BAD_CU_SEQLENS, CMR_ECUDA, CMR_EINVAL, CMR_EUNSUPPORTED, CMR_OK,
+                  CmrError, lib, positions, positions_step, rotate_qk, version)
+
+__all__ = ["positions", "positions_step", "rotate_qk", "lib", "version", "CmrError",
+           "CMR_OK", "CMR_EINVAL", "CMR_ECUDA", "CMR_EUNSUPPORTED", "CMR_DEVICE_BAD_CU_SEQLENS"]

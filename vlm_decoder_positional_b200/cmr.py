@@ -1,0 +1,190 @@
+"""Python binding of libcmr (include/cmr.h): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels; this module checks
+tensor dtypes/devices/shapes, allocates outputs with torch when the caller does
+not pass them, and forwards raw pointers and the current CUDA stream.  There
+is no fallback: if libcmr.so is missing or a call fails, it raises.
+"""
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcmr.so")
+
+CMR_OK, CMR_EINVAL, CMR_ECUDA, CMR_EUNSUPPORTED = 0, 1, 2, 3
+CMR_DEVICE_BAD_CU_SEQLENS = 1
+
+IMAGE_TOKEN_ID = 248078
+
+# name -> (restype, argtypes); mirrors include/cmr.h
+_i32p = ctypes.c_void_p
+SIGNATURES = {
+    "cmr_positions": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                     _i32p, _i32p, _i32p, _i32p, ctypes.c_void_p]),
+    "cmr_positions_step": (ctypes.c_int, [_i32p, _i32p, _i32p, ctypes.c_int32, _i32p,
+                                          ctypes.c_void_p]),
+    "cmr_rotate_qk": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p, ctypes.c_int64,
+                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.c_double,
+                                     ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                     ctypes.c_void_p]),
+    "cmr_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "cmr_last_error_message": (ctypes.c_char_p, []),
+    "cmr_version": (ctypes.c_int32, []),
+}
+
+_lib = None
+
+
+class CmrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().cmr_last_error_message().decode()
+        super().__init__(f"{where}: {lib().cmr_status_string(status).decode()} -- {msg}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libcmr.so with its signatures set; raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m vlm_decoder_positional_b200.build`"
+                " (there is no CPU fallback)")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def version() -> int:
+    return int(lib().cmr_version())
+
+
+def _check(status: int, where: str):
+    if status != CMR_OK:
+        raise CmrError(status, where)
+
+
+def _stream_ptr(device: torch.device, stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return int(s.cuda_stream)
+
+
+def _want(t: torch.Tensor, name: str, dtype: torch.dtype, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def positions(ids: torch.Tensor, cu_seqlens: torch.Tensor, image_token_id: int = IMAGE_TOKEN_ID,
+              out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+              device_status: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None):
+    """cmr_positions: (pos int32 [3, N], start int32 [B], amount int32 [B])."""
+    _want(ids, "ids", torch.int32)
+    _want(cu_seqlens, "cu_seqlens", torch.int32, ids.device)
+    n, b = ids.numel(), cu_seqlens.numel() - 1
+    if b < 0:
+        raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+    if out is None:
+        pos = torch.empty((3, n), dtype=torch.int32, device=ids.device)
+        start = torch.empty(b, dtype=torch.int32, device=ids.device)
+        amount = torch.empty(b, dtype=torch.int32, device=ids.device)
+    else:
+        pos, start, amount = out
+        _want(pos, "pos", torch.int32, ids.device)
+        _want(start, "start", torch.int32, ids.device)
+        _want(amount, "amount", torch.int32, ids.device)
+        if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
+            raise ValueError("output shapes must be [3, N], [B], [B]")
+    st_ptr = None
+    if device_status is not None:
+        _want(device_status, "device_status", torch.int32, ids.device)
+        st_ptr = device_status.data_ptr()
+    with torch.cuda.device(ids.device):
+        _check(lib().cmr_positions(ids.data_ptr() if n else None, cu_seqlens.data_ptr(), b, n,
+                                   int(image_token_id), pos.data_ptr() if n else None,
+                                   start.data_ptr() if b else None,
+                                   amount.data_ptr() if b else None, st_ptr,
+                                   _stream_ptr(ids.device, stream)), "cmr_positions")
+    return pos, start, amount
+
+
+def positions_step(cache_len: torch.Tensor, start: torch.Tensor, amount: torch.Tensor,
+                   out: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """cmr_positions_step: pos int32 [3, B] of the token at index cache_len[b]."""
+    _want(cache_len, "cache_len", torch.int32)
+    _want(start, "start", torch.int32, cache_len.device)
+    _want(amount, "amount", torch.int32, cache_len.device)
+    b = cache_len.numel()
+    if start.numel() != b or amount.numel() != b:
+        raise ValueError("cache_len, start and amount must have the same length")
+    pos = out if out is not None else torch.empty((3, b), dtype=torch.int32,
+                                                  device=cache_len.device)
+    _want(pos, "out", torch.int32, cache_len.device)
+    if pos.shape != (3, b):
+        raise ValueError("out must be [3, B]")
+    if b == 0:
+        return pos
+    with torch.cuda.device(cache_len.device):
+        _check(lib().cmr_positions_step(cache_len.data_ptr(), start.data_ptr(), amount.data_ptr(),
+                                        b, pos.data_ptr(),
+                                        _stream_ptr(cache_len.device, stream)),
+               "cmr_positions_step")
+    return pos
+
+
+def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor,
+              theta: float = 1e7, sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
+              stream: Optional[torch.cuda.Stream] = None):
+    """cmr_rotate_qk, in place.  q: bf16 [L, N, hq, D] (or [N, hq, D]); k likewise
+    with hk heads; pos: int32 [3, N].  Returns (q, k)."""
+    _want(pos, "pos", torch.int32)
+    dev = pos.device
+    if pos.dim() != 2 or pos.shape[0] != 3:
+        raise ValueError("pos must be [3, N]")
+    n = pos.shape[1]
+
+    def shape_of(t, name):
+        if t is None:
+            return None
+        _want(t, name, torch.bfloat16, dev)
+        if t.dim() == 3:
+            return (1,) + tuple(t.shape)
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [L, N, H, D] or [N, H, D]")
+        return tuple(t.shape)
+
+    qs, ks = shape_of(q, "q"), shape_of(k, "k")
+    if qs is None and ks is None:
+        raise ValueError("need q or k")
+    ref = qs or ks
+    L, D = ref[0], ref[3]
+    for s, name in ((qs, "q"), (ks, "k")):
+        if s is not None and (s[0] != L or s[1] != n or s[3] != D):
+            raise ValueError(f"{name} shape {s} does not match L={L}, N={n}, D={D}")
+    hq = qs[2] if qs else 0
+    hk = ks[2] if ks else 0
+    sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
+    with torch.cuda.device(dev):
+        _check(lib().cmr_rotate_qk(q.data_ptr() if q is not None and q.numel() else None,
+                                   k.data_ptr() if k is not None and k.numel() else None,
+                                   pos.data_ptr() if n else None, n, L, hq, hk, D, float(theta),
+                                   sec, int(rot_dim), _stream_ptr(dev, stream)),
+               "cmr_rotate_qk")
+    return q, k

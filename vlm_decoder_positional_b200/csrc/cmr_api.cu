@@ -1,0 +1,180 @@
+// The C ABI of libcmr (declared in include/cmr.h): host-side argument checks,
+// the per-frequency tables, and the kernel launches.  Nothing here allocates
+// device memory or synchronises.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+
+#include "cmr.h"
+#include "cmr_internal.cuh"
+
+namespace {
+
+thread_local char g_message[320] = "no error";
+
+cmr_status fail(cmr_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_message, sizeof g_message, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+cmr_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(CMR_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// A pointer the current device can use in a kernel: device or managed memory
+// of the current device.  Pageable host memory would fault in a kernel, so it
+// is refused here.
+cmr_status check_device_ptr(const void* p, const char* name) {
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();  // clear the error this query may have set
+    return fail(CMR_EINVAL, "%s: not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+  }
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+    return fail(CMR_EINVAL, "%s: not device memory (memory type %d)", name,
+                static_cast<int>(attr.type));
+  int dev = -1;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (attr.type == cudaMemoryTypeDevice && attr.device != dev)
+    return fail(CMR_EINVAL, "%s: lives on device %d but device %d is current", name,
+                attr.device, dev);
+  return CMR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* cmr_status_string(cmr_status s) {
+  switch (s) {
+    case CMR_OK: return "CMR_OK";
+    case CMR_EINVAL: return "CMR_EINVAL: invalid argument";
+    case CMR_ECUDA: return "CMR_ECUDA: CUDA runtime error";
+    case CMR_EUNSUPPORTED: return "CMR_EUNSUPPORTED: shape outside this build's limits";
+  }
+  return "unknown cmr_status";
+}
+
+const char* cmr_last_error_message(void) { return g_message; }
+
+int32_t cmr_version(void) { return 10000; }  // 1.0.0
+
+cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                         int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
+                         int32_t* out_start, int32_t* out_amount, int32_t* device_status,
+                         cmr_stream_t stream) {
+  if (num_seqs < 0 || n_tokens < 0) return fail(CMR_EINVAL, "negative num_seqs or n_tokens");
+  if (n_tokens > INT32_MAX) return fail(CMR_EINVAL, "n_tokens exceeds int32 indexing");
+  if (num_seqs == 0) {
+    if (n_tokens != 0) return fail(CMR_EINVAL, "num_seqs == 0 with n_tokens > 0");
+    return CMR_OK;
+  }
+  if (!cu_seqlens || !out_start || !out_amount)
+    return fail(CMR_EINVAL, "cu_seqlens, out_start and out_amount are required");
+  if (n_tokens > 0 && (!ids || !out_pos)) return fail(CMR_EINVAL, "ids and out_pos are required");
+  cmr_status s;
+  if ((s = check_device_ptr(cu_seqlens, "cu_seqlens")) != CMR_OK) return s;
+  if ((s = check_device_ptr(out_start, "out_start")) != CMR_OK) return s;
+  if ((s = check_device_ptr(out_amount, "out_amount")) != CMR_OK) return s;
+  if (n_tokens > 0) {
+    if ((s = check_device_ptr(ids, "ids")) != CMR_OK) return s;
+    if ((s = check_device_ptr(out_pos, "out_pos")) != CMR_OK) return s;
+  }
+  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
+                                        out_pos, out_start, out_amount, device_status,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* start,
+                              const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
+                              cmr_stream_t stream) {
+  if (num_seqs < 0) return fail(CMR_EINVAL, "negative num_seqs");
+  if (num_seqs == 0) return CMR_OK;
+  if (!cache_len || !start || !amount || !out_pos)
+    return fail(CMR_EINVAL, "cache_len, start, amount and out_pos are required");
+  cmr_status s;
+  if ((s = check_device_ptr(cache_len, "cache_len")) != CMR_OK) return s;
+  if ((s = check_device_ptr(start, "start")) != CMR_OK) return s;
+  if ((s = check_device_ptr(amount, "amount")) != CMR_OK) return s;
+  if ((s = check_device_ptr(out_pos, "out_pos")) != CMR_OK) return s;
+  cudaError_t e = cmr::launch_positions_step(cache_len, start, amount, num_seqs, out_pos,
+                                             reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions_step launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
+                         int32_t num_layers, int32_t hq, int32_t hk, int32_t head_dim,
+                         double theta, const int32_t sections[3], int32_t rot_dim,
+                         cmr_stream_t stream) {
+  if (n_tokens < 0 || num_layers < 0) return fail(CMR_EINVAL, "negative n_tokens or num_layers");
+  if (hq < 0 || hk < 0 || hq + hk < 1) return fail(CMR_EINVAL, "need hq, hk >= 0, hq + hk >= 1");
+  if (head_dim <= 0 || head_dim % 8 != 0) return fail(CMR_EINVAL, "head_dim must be a positive multiple of 8");
+  if (rot_dim < 16 || rot_dim % 16 != 0 || rot_dim > head_dim || rot_dim > 2 * cmr::kMaxFreqs)
+    return fail(CMR_EINVAL, "rot_dim must be a multiple of 16 in [16, min(head_dim, 256)]");
+  if (!(theta > 0.0) || !std::isfinite(theta)) return fail(CMR_EINVAL, "theta must be finite and > 0");
+  if (!sections) return fail(CMR_EINVAL, "sections is required");
+
+  // Frequency -> plane: H takes j = 1, 4, 7, ... (sections[1] of them), W takes
+  // j = 2, 5, 8, ... (sections[2]), T keeps the rest and must count sections[0].
+  const int F = rot_dim / 2;
+  cmr::FreqTable table;
+  for (int j = 0; j < cmr::kMaxFreqs; ++j) {
+    table.plane[j] = 0;
+    table.inv_freq[j] = 0.0;
+  }
+  if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
+      static_cast<int64_t>(sections[0]) + sections[1] + sections[2] != F)
+    return fail(CMR_EINVAL, "sections must be >= 0 and sum to rot_dim / 2");
+  for (int plane = 1; plane <= 2; ++plane)
+    for (int m = 0; m < sections[plane]; ++m) {
+      const int j = 3 * m + plane;
+      if (j >= F) return fail(CMR_EINVAL, "sections[%d] = %d does not fit the interleave", plane, sections[plane]);
+      table.plane[j] = plane;
+    }
+  for (int j = 0; j < F; ++j) table.inv_freq[j] = std::pow(theta, -2.0 * j / rot_dim);
+
+  const int units_per_head = rot_dim / 16;
+  const int64_t units = static_cast<int64_t>(hq + hk) * units_per_head;
+  if (units > cmr::kMaxUnitsPerToken)
+    return fail(CMR_EUNSUPPORTED, "(hq + hk) * rot_dim / 16 = %lld exceeds %d",
+                static_cast<long long>(units), cmr::kMaxUnitsPerToken);
+  if (n_tokens == 0 || num_layers == 0) return CMR_OK;
+  if (!pos) return fail(CMR_EINVAL, "pos is required");
+  if (hq > 0 && !q) return fail(CMR_EINVAL, "q is required when hq > 0");
+  if (hk > 0 && !k) return fail(CMR_EINVAL, "k is required when hk > 0");
+  if ((hq > 0 && !aligned16(q)) || (hk > 0 && !aligned16(k)))
+    return fail(CMR_EINVAL, "q and k must be 16-byte aligned");
+  cmr_status s;
+  if ((s = check_device_ptr(pos, "pos")) != CMR_OK) return s;
+  if (hq > 0 && (s = check_device_ptr(q, "q")) != CMR_OK) return s;
+  if (hk > 0 && (s = check_device_ptr(k, "k")) != CMR_OK) return s;
+
+  cmr::RotateArgs a{};
+  a.q = static_cast<uint16_t*>(q);
+  a.k = static_cast<uint16_t*>(k);
+  a.pos = pos;
+  a.n_tokens = n_tokens;
+  a.num_layers = num_layers;
+  a.hq = hq;
+  a.hk = hk;
+  a.head_dim = head_dim;
+  a.rot_dim = rot_dim;
+  a.units_per_head = units_per_head;
+  a.units_per_token = static_cast<int32_t>(units);
+  cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
+  return CMR_OK;
+}
+
+}  // extern "C"

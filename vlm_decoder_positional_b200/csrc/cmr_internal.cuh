@@ -1,0 +1,60 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libcmr.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cmr.h"
+
+namespace cmr {
+
+// ---- canvas geometry of one 448x448 image (HF card "How the VLM rides the
+// text-only engine": 64 merged rows on an 8x8 grid, framed by <image> and
+// </image>, followed by the template's "\n") ----
+constexpr int kGridSide = 8;
+constexpr int kGridRows = kGridSide * kGridSide;   // 64
+constexpr int kFrameTokens = kGridRows + 3;        // <image>, rows, </image>, "\n" = 67
+constexpr int kCanvasSpan = kGridSide + 1;         // max(H, W) + 1 = 9
+constexpr int32_t kTextOnlyStart = 1 << 30;
+
+// ---- rotation limits ----
+constexpr int kMaxFreqs = 128;          // rot_dim <= 256
+constexpr int kMaxUnitsPerToken = 512;  // (hq + hk) * rot_dim / 16 = threads per token
+
+// Per-frequency tables, passed by value as a kernel parameter (1.2 KB) and
+// staged into shared memory by each CTA.
+struct FreqTable {
+  double inv_freq[kMaxFreqs];
+  int32_t plane[kMaxFreqs];
+};
+
+struct RotateArgs {
+  uint16_t* q;  // bf16 bits [L, N, hq, D]
+  uint16_t* k;  // bf16 bits [L, N, hk, D]
+  const int32_t* pos;  // [3, N]
+  int64_t n_tokens;
+  int32_t num_layers;
+  int32_t hq, hk, head_dim, rot_dim;
+  int32_t units_per_head;   // rot_dim / 16: 8-dim chunks of the first half
+  int32_t units_per_token;  // (hq + hk) * units_per_head
+  int32_t slots;            // token slots per CTA
+  int32_t group;            // tokens per slot per tile
+};
+
+struct LaunchShape {
+  dim3 grid, block;
+  size_t smem;
+};
+
+cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                             int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
+                             int32_t* out_start, int32_t* out_amount, int32_t* device_status,
+                             cudaStream_t stream);
+
+cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start,
+                                  const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
+                                  cudaStream_t stream);
+
+cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream);
+
+}  // namespace cmr
