@@ -132,7 +132,7 @@ CMR_API cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* s
  *          rot_dim / 2, each realisable by the interleave above
  *   rot_dim   multiple of 16, 16 .. min(head_dim, 256)  (64 for this model)
  * Errors: CMR_EINVAL for any violation above; CMR_EUNSUPPORTED when
- * (hq + hk) * rot_dim / 16 > 512. */
+ * (hq + hk) * num_layers > INT32_MAX. */
 CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
                          int32_t num_layers, int32_t hq, int32_t hk,
                          int32_t head_dim, double theta,

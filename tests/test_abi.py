@@ -72,8 +72,8 @@ def test_rotate_rejects_bad_arguments_on_the_host(lib, kw):
     assert lib.cmr_last_error_message()
 
 
-def test_rotate_too_many_heads_is_unsupported(lib):
-    st = lib.cmr_rotate_qk(FAKE, FAKE, FAKE, 10, 1, 100, 29, 256, 1e7, SEC, 64, None)
+def test_rotate_too_many_head_rows_is_unsupported(lib):
+    st = lib.cmr_rotate_qk(FAKE, FAKE, FAKE, 10, 80000, 30000, 2, 256, 1e7, SEC, 64, None)
     assert st == cmr.CMR_EUNSUPPORTED
 
 

@@ -3,6 +3,7 @@
 // device memory or synchronises.
 #include <cmath>
 #include <cstdarg>
+#include <climits>
 #include <cstdio>
 
 #include "cmr.h"
@@ -144,11 +145,10 @@ cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
     }
   for (int j = 0; j < F; ++j) table.inv_freq[j] = std::pow(theta, -2.0 * j / rot_dim);
 
-  const int units_per_head = rot_dim / 16;
-  const int64_t units = static_cast<int64_t>(hq + hk) * units_per_head;
-  if (units > cmr::kMaxUnitsPerToken)
-    return fail(CMR_EUNSUPPORTED, "(hq + hk) * rot_dim / 16 = %lld exceeds %d",
-                static_cast<long long>(units), cmr::kMaxUnitsPerToken);
+  const int64_t rows = (static_cast<int64_t>(hq) + hk) * num_layers;  // head rows per token
+  if (rows > INT32_MAX)
+    return fail(CMR_EUNSUPPORTED, "(hq + hk) * num_layers = %lld exceeds INT32_MAX",
+                static_cast<long long>(rows));
   if (n_tokens == 0 || num_layers == 0) return CMR_OK;
   if (!pos) return fail(CMR_EINVAL, "pos is required");
   if (hq > 0 && !q) return fail(CMR_EINVAL, "q is required when hq > 0");
@@ -170,8 +170,7 @@ cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
   a.hk = hk;
   a.head_dim = head_dim;
   a.rot_dim = rot_dim;
-  a.units_per_head = units_per_head;
-  a.units_per_token = static_cast<int32_t>(units);
+  a.units_per_head = rot_dim / 16;
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
   return CMR_OK;

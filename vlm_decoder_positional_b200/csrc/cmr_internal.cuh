@@ -18,8 +18,7 @@ constexpr int kCanvasSpan = kGridSide + 1;         // max(H, W) + 1 = 9
 constexpr int32_t kTextOnlyStart = 1 << 30;
 
 // ---- rotation limits ----
-constexpr int kMaxFreqs = 128;          // rot_dim <= 256
-constexpr int kMaxUnitsPerToken = 512;  // (hq + hk) * rot_dim / 16 = threads per token
+constexpr int kMaxFreqs = 128;  // rot_dim <= 256
 
 // Per-frequency tables, passed by value as a kernel parameter (1.2 KB) and
 // staged into shared memory by each CTA.
@@ -35,15 +34,7 @@ struct RotateArgs {
   int64_t n_tokens;
   int32_t num_layers;
   int32_t hq, hk, head_dim, rot_dim;
-  int32_t units_per_head;   // rot_dim / 16: 8-dim chunks of the first half
-  int32_t units_per_token;  // (hq + hk) * units_per_head
-  int32_t slots;            // token slots per CTA
-  int32_t group;            // tokens per slot per tile
-};
-
-struct LaunchShape {
-  dim3 grid, block;
-  size_t smem;
+  int32_t units_per_head;  // rot_dim / 16: threads per token, 8 frequencies each
 };
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,

@@ -6,20 +6,22 @@
 // of F = rot_dim/2 reads the position of its plane, a = pos[plane_j][t] *
 // theta^(-2j/rot_dim), and turns the pair (x_j, x_{j+F}) of every head.
 //
-// Memory: the op touches rot_dim of head_dim dims per head (128 B of every
-// 512-B head row for this model) and is bound by HBM.  Each thread owns one
-// "unit" = 8 consecutive dims of the first half plus their 8 partners of the
-// second half of one head: two 16-byte loads and two 16-byte stores, the pair
-// partner in the same thread, no shuffles.  Four consecutive lanes cover one
-// head's 64 B + 64 B, so every warp access covers whole 32-B sectors.
+// The op touches rot_dim of head_dim dims per head (128 B of every 512-B head
+// row for this model), reads and writes each byte once, and is bound by HBM;
+// it is not a contraction, so there are no tensor cores here.
 //
-// Per tile of tokens, a CTA first computes cos/sin for every (token,
-// frequency) once -- fp64 angle and fp64 reduction modulo 2*pi, fp32 sincos --
-// into shared memory, then applies it to every head of Q and K of every layer
-// (num_layers layers share pos).  Up to kJobs (token, layer) jobs per thread
-// are loaded before any is computed, which keeps 8 x 32 B in flight per
-// thread.  The grid is persistent: one wave of CTAs at full occupancy on all
-// SMs striding over tiles.
+// Thread map: a token's rotated dims split into U = rot_dim/16 "units" of 8
+// frequencies; thread (t, u) owns dims [8u, 8u+8) and their partners
+// [F+8u, F+8u+8) of token t in every head of Q and K and every layer.  It
+// computes the cos/sin of its 8 frequencies once (fp64 angle, fp64 reduction
+// modulo 2*pi, fp32 sincos) and reuses them for all (hq + hk) * num_layers
+// head rows, so each (token, frequency) pair is evaluated exactly once and no
+// thread waits on another: there is no shared cos/sin table and no barrier
+// in the loop.  Lanes 4t'..4t'+3 of a warp hold one token, so every warp access
+// is 8 tokens x 64 contiguous bytes (whole 32-B sectors), and the x / partner
+// loads of one head row together cover its 128-B line.  kBatch head rows are
+// loaded (two 16-byte loads each, evict-first) before any is rotated and
+// stored back (two 16-byte stores each).
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -29,25 +31,26 @@
 namespace cmr {
 namespace {
 
-constexpr int kJobs = 8;          // (token, layer) jobs in flight per thread
-constexpr int kMaxThreads = 512;  // CTA size bound (slots * units_per_token)
+constexpr int kThreads = 256;
+constexpr int kMinBlocksPerSm = 2;
+constexpr int kBatch = 4;  // head rows in flight per thread
 
 // 2*pi split in two doubles (Cody & Waite's additive range reduction):
 // kTwoPiHi is 2*pi rounded to double and kTwoPiLo the rounding remainder.
 constexpr double kTwoPiHi = 6.283185307179586232e+00;
 constexpr double kTwoPiLo = 2.449293598294706414e-16;
 constexpr double kInvTwoPi = 1.591549430918953358e-01;
+constexpr double kInvPi = 3.183098861837906715e-01;
 
-// cos/sin of p * inv_freq: the product and its reduction to [-pi, pi] in
-// fp64 (exact to ~1e-16 relative for |p| < 2^31), then fp32 sincos.
-__device__ __forceinline__ float2 cos_sin(int32_t p, double inv_freq) {
+// cos/sin of p * inv_freq: the product and its reduction to r in [-pi, pi] in
+// fp64 (absolute error ~1e-16 for |p| < 2^31), then sincospif(r / pi) in fp32,
+// whose own reduction of an argument in [-1, 1] is exact.
+__device__ __forceinline__ void cos_sin(int32_t p, double inv_freq, float& c, float& s) {
   const double a = static_cast<double>(p) * inv_freq;
   const double n = rint(a * kInvTwoPi);
   double r = fma(-n, kTwoPiHi, a);
   r = fma(-n, kTwoPiLo, r);
-  float s, c;
-  sincosf(static_cast<float>(r), &s, &c);
-  return make_float2(c, s);
+  sincospif(static_cast<float>(r * kInvPi), &s, &c);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -58,178 +61,134 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Rotate one unit: x1 = dims [8u, 8u+8), x2 = their partners [F+8u, F+8u+8).
-// cs points at the 8 (cos, sin) pairs of those frequencies in shared memory.
-__device__ __forceinline__ void rotate_unit(uint4& x1, uint4& x2, const float2* __restrict__ cs) {
-  const float4* c4 = reinterpret_cast<const float4*>(cs);
+// Rotate one unit: x1 holds dims [8u, 8u+8), x2 their partners [F+8u, F+8u+8).
+__device__ __forceinline__ void rotate_unit(uint4& x1, uint4& x2, const float (&c)[8],
+                                            const float (&s)[8]) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&x1);
   uint32_t* b = reinterpret_cast<uint32_t*>(&x2);
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const float4 t = c4[m];  // (cos, sin) of frequencies 2m and 2m+1 of the unit
     const float a0 = bf16_lo(a[m]), a1 = bf16_hi(a[m]);
     const float b0 = bf16_lo(b[m]), b1 = bf16_hi(b[m]);
-    const float y0 = a0 * t.x - b0 * t.y;
-    const float z0 = b0 * t.x + a0 * t.y;
-    const float y1 = a1 * t.z - b1 * t.w;
-    const float z1 = b1 * t.z + a1 * t.w;
-    a[m] = pack_bf16x2(y0, y1);
-    b[m] = pack_bf16x2(z0, z1);
+    const float c0 = c[2 * m], s0 = s[2 * m], c1 = c[2 * m + 1], s1 = s[2 * m + 1];
+    a[m] = pack_bf16x2(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
+    b[m] = pack_bf16x2(b0 * c0 + a0 * s0, b1 * c1 + a1 * s1);
   }
 }
 
-__global__ void __launch_bounds__(kMaxThreads)
+__global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
     rotate_qk_kernel(const RotateArgs args, const FreqTable table) {
-  extern __shared__ float4 s_dyn[];
-  float2* s_cs = reinterpret_cast<float2*>(s_dyn);  // [slots * group][F]
   __shared__ double s_inv[kMaxFreqs];
   __shared__ int32_t s_plane[kMaxFreqs];
-
   const int F = args.rot_dim >> 1;
   for (int j = threadIdx.x; j < F; j += blockDim.x) {
     s_inv[j] = table.inv_freq[j];
     s_plane[j] = table.plane[j];
   }
+  __syncthreads();  // the only barrier: the tables are read-only from here on
 
-  // Fixed role of this thread inside its token slot.
-  const int W = args.units_per_token;
   const int U = args.units_per_head;
-  const int slot = threadIdx.x / W;
-  const int w = threadIdx.x - slot * W;
-  const int head = w / U;
-  const int unit = w - head * U;
-  const bool active = slot < args.slots;
-  const bool is_q = head < args.hq;
-  uint16_t* const base = is_q ? args.q : args.k;
-  const int64_t heads_here = is_q ? args.hq : args.hk;
-  const int64_t head_idx = is_q ? head : head - args.hq;
-  const int64_t tok_stride = heads_here * args.head_dim;
-  const int64_t layer_stride = args.n_tokens * tok_stride;
-  const int64_t unit_off = head_idx * args.head_dim + unit * 8;
+  const int tokens_per_cta = kThreads / U;
+  const int local = threadIdx.x / U;
+  const int u = threadIdx.x - local * U;
+  if (local >= tokens_per_cta) return;  // spare threads when U does not divide kThreads
 
-  const int L = args.num_layers;
-  const int G = args.group;
-  const int tile_tokens = args.slots * G;
-  const int jobs = G * L;
-  const int64_t n_tiles = (args.n_tokens + tile_tokens - 1) / tile_tokens;
-  __syncthreads();
+  const int64_t N = args.n_tokens;
+  const int H = args.hq + args.hk;
+  const int J = H * args.num_layers;  // head rows per token
+  const int64_t D = args.head_dim;
+  const int64_t q_tok = static_cast<int64_t>(args.hq) * D;  // elements per token
+  const int64_t k_tok = static_cast<int64_t>(args.hk) * D;
+  const int64_t q_layer = N * q_tok;
+  const int64_t k_layer = N * k_tok;
+  const int half4 = F / 8;  // partner offset in 16-byte vectors
 
-  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int64_t t0 = tile * tile_tokens;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * tokens_per_cta + local; t < N;
+       t += static_cast<int64_t>(gridDim.x) * tokens_per_cta) {
+    // Base of this thread's unit in head 0 of layer 0; K rows are indexed by
+    // h - hq, folded into the base so that row h sits at base + h * D.
+    uint16_t* const q_base = args.q + t * q_tok + 8 * u;
+    uint16_t* const k_base = args.k + t * k_tok + 8 * u - static_cast<int64_t>(args.hq) * D;
 
-    // Phase 1: cos/sin of every (token, frequency) in the tile.
-    for (int idx = threadIdx.x; idx < tile_tokens * F; idx += blockDim.x) {
-      const int lt = idx / F;
-      const int j = idx - lt * F;
-      const int64_t t = t0 + lt;
-      float2 v = make_float2(1.f, 0.f);
-      if (t < args.n_tokens) v = cos_sin(__ldg(args.pos + s_plane[j] * args.n_tokens + t), s_inv[j]);
-      s_cs[idx] = v;
+    // cos/sin of the unit's 8 frequencies at token t.
+    const int32_t p0 = __ldg(args.pos + t);
+    const int32_t p1 = __ldg(args.pos + N + t);
+    const int32_t p2 = __ldg(args.pos + 2 * N + t);
+    float c[8], s[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = 8 * u + e;
+      const int pl = s_plane[j];
+      cos_sin(pl == 0 ? p0 : (pl == 1 ? p1 : p2), s_inv[j], c[e], s[e]);
     }
-    __syncthreads();
 
-    // Phase 2: every head of Q and K, every layer, of the slot's G tokens.
-    if (active) {
-      const int64_t slot_t0 = t0 + static_cast<int64_t>(slot) * G;
-      for (int jb = 0; jb < jobs; jb += kJobs) {
-        uint4 x1[kJobs], x2[kJobs];
-        int gi[kJobs];
-        bool ok[kJobs];
-        int g = jb / L, l = jb - (jb / L) * L;
+    int h = 0, l = 0;  // head row of the next job: head h of layer l
+    for (int j0 = 0; j0 < J; j0 += kBatch) {
+      uint4 x1[kBatch], x2[kBatch];
+      uint4* ptr[kBatch];
 #pragma unroll
-        for (int x = 0; x < kJobs; ++x) {
-          gi[x] = g;
-          ok[x] = (jb + x < jobs) && (slot_t0 + g < args.n_tokens);
-          if (ok[x]) {
-            const uint4* p = reinterpret_cast<const uint4*>(
-                base + l * layer_stride + (slot_t0 + g) * tok_stride + unit_off);
-            x1[x] = __ldcs(p);
-            x2[x] = __ldcs(reinterpret_cast<const uint4*>(
-                reinterpret_cast<const uint16_t*>(p) + F));
-          }
-          if (++l == L) {
-            l = 0;
-            ++g;
-          }
-        }
-        g = jb / L;
-        l = jb - g * L;
-#pragma unroll
-        for (int x = 0; x < kJobs; ++x) {
-          if (ok[x]) {
-            const float2* cs = s_cs + (slot * G + gi[x]) * F + unit * 8;
-            rotate_unit(x1[x], x2[x], cs);
-            uint4* p = reinterpret_cast<uint4*>(base + l * layer_stride +
-                                                (slot_t0 + g) * tok_stride + unit_off);
-            __stcs(p, x1[x]);
-            __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p) + F), x2[x]);
-          }
-          if (++l == L) {
-            l = 0;
-            ++g;
+      for (int b = 0; b < kBatch; ++b) {
+        ptr[b] = nullptr;
+        if (j0 + b < J) {
+          uint16_t* row = (h < args.hq) ? q_base + l * q_layer : k_base + l * k_layer;
+          ptr[b] = reinterpret_cast<uint4*>(row + h * D);
+          x1[b] = __ldcs(ptr[b]);
+          x2[b] = __ldcs(ptr[b] + half4);
+          if (++h == H) {
+            h = 0;
+            ++l;
           }
         }
       }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        if (ptr[b] != nullptr) {
+          rotate_unit(x1[b], x2[b], c, s);
+          __stcs(ptr[b], x1[b]);
+          __stcs(ptr[b] + half4, x2[b]);
+        }
+      }
     }
-    __syncthreads();  // s_cs is rewritten by the next tile
   }
 }
 
 struct OccupancyCache {
   std::mutex mu;
   int device = -1;
-  int sms = 0;
-  int threads = 0;
-  size_t smem = 0;
-  int blocks_per_sm = 0;
+  int ctas = 0;
 };
 OccupancyCache g_occ[64];
 
-cudaError_t resident_ctas(int threads, size_t smem, int* total) {
+// CTAs resident on the whole device at full occupancy (cached per device).
+cudaError_t resident_ctas(int* total) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   OccupancyCache& c = g_occ[dev & 63];
   std::lock_guard<std::mutex> lock(c.mu);
-  if (c.device != dev || c.threads != threads || c.smem != smem) {
+  if (c.device != dev) {
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_qk_kernel, threads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_qk_kernel, kThreads, 0);
     if (e != cudaSuccess) return e;
     c.device = dev;
-    c.sms = sms;
-    c.threads = threads;
-    c.smem = smem;
-    c.blocks_per_sm = per_sm > 0 ? per_sm : 1;
+    c.ctas = sms * (per_sm > 0 ? per_sm : 1);
   }
-  *total = c.sms * c.blocks_per_sm;
+  *total = c.ctas;
   return cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream) {
-  RotateArgs a = in;
-  const int W = a.units_per_token;
-  // Token slots per CTA: as many whole tokens as fit in 320 threads (8 for
-  // 8 Q + 2 K heads at rot_dim 64), at least one.
-  int slots = 320 / W;
-  if (slots < 1) slots = 1;
-  if (slots > 32) slots = 32;
-  a.slots = slots;
-  // Tokens per slot per tile: enough (token, layer) jobs to fill kJobs.
-  int group = kJobs / (a.num_layers > 0 ? a.num_layers : 1);
-  a.group = group < 1 ? 1 : group;
-  const int threads = ((slots * W + 31) / 32) * 32;
-  const size_t smem = sizeof(float2) * static_cast<size_t>(slots) * a.group * (a.rot_dim / 2);
+cudaError_t launch_rotate_qk(const RotateArgs& a, const FreqTable& table, cudaStream_t stream) {
   int max_ctas = 0;
-  cudaError_t e = resident_ctas(threads, smem, &max_ctas);
+  cudaError_t e = resident_ctas(&max_ctas);
   if (e != cudaSuccess) return e;
-  const int64_t tile_tokens = static_cast<int64_t>(slots) * a.group;
-  const int64_t n_tiles = (a.n_tokens + tile_tokens - 1) / tile_tokens;
-  const int64_t ctas = n_tiles < max_ctas ? n_tiles : max_ctas;
-  rotate_qk_kernel<<<static_cast<unsigned>(ctas), threads, smem, stream>>>(a, table);
+  const int64_t tokens_per_cta = kThreads / a.units_per_head;
+  const int64_t needed = (a.n_tokens + tokens_per_cta - 1) / tokens_per_cta;
+  const int64_t ctas = needed < max_ctas ? needed : max_ctas;
+  rotate_qk_kernel<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
   return cudaGetLastError();
 }
 
