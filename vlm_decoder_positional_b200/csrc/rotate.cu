@@ -31,8 +31,8 @@
 namespace cmr {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kMinBlocksPerSm = 2;
+constexpr int kThreads = 128;
+constexpr int kMinBlocksPerSm = 4;
 constexpr int kBatch = 4;  // head rows in flight per thread
 
 // 2*pi split in two doubles (Cody & Waite's additive range reduction):
@@ -103,29 +103,27 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
   const int64_t k_layer = N * k_tok;
   const int half4 = F / 8;  // partner offset in 16-byte vectors
 
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * tokens_per_cta + local; t < N;
-       t += static_cast<int64_t>(gridDim.x) * tokens_per_cta) {
+  const int64_t t_step = static_cast<int64_t>(gridDim.x) * tokens_per_cta;
+  int64_t t = static_cast<int64_t>(blockIdx.x) * tokens_per_cta + local;
+  // Planes of the current token, loaded one token ahead so that their latency
+  // overlaps the previous token's head rows.
+  int32_t p0 = 0, p1 = 0, p2 = 0;
+  if (t < N) {
+    p0 = __ldg(args.pos + t);
+    p1 = __ldg(args.pos + N + t);
+    p2 = __ldg(args.pos + 2 * N + t);
+  }
+  for (; t < N; t += t_step) {
     // Base of this thread's unit in head 0 of layer 0; K rows are indexed by
     // h - hq, folded into the base so that row h sits at base + h * D.
     uint16_t* const q_base = args.q + t * q_tok + 8 * u;
     uint16_t* const k_base = args.k + t * k_tok + 8 * u - static_cast<int64_t>(args.hq) * D;
 
-    // cos/sin of the unit's 8 frequencies at token t.
-    const int32_t p0 = __ldg(args.pos + t);
-    const int32_t p1 = __ldg(args.pos + N + t);
-    const int32_t p2 = __ldg(args.pos + 2 * N + t);
-    float c[8], s[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int j = 8 * u + e;
-      const int pl = s_plane[j];
-      cos_sin(pl == 0 ? p0 : (pl == 1 ? p1 : p2), s_inv[j], c[e], s[e]);
-    }
-
+    // First batch of head rows in flight before the cos/sin work below.
     int h = 0, l = 0;  // head row of the next job: head h of layer l
-    for (int j0 = 0; j0 < J; j0 += kBatch) {
-      uint4 x1[kBatch], x2[kBatch];
-      uint4* ptr[kBatch];
+    uint4 x1[kBatch], x2[kBatch];
+    uint4* ptr[kBatch];
+    auto load_batch = [&](int j0) {
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
         ptr[b] = nullptr;
@@ -140,6 +138,25 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
           }
         }
       }
+    };
+    load_batch(0);
+
+    // cos/sin of the unit's 8 frequencies at token t.
+    float c[8], s[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = 8 * u + e;
+      const int pl = s_plane[j];
+      cos_sin(pl == 0 ? p0 : (pl == 1 ? p1 : p2), s_inv[j], c[e], s[e]);
+    }
+    const int64_t tn = t + t_step;
+    if (tn < N) {
+      p0 = __ldg(args.pos + tn);
+      p1 = __ldg(args.pos + N + tn);
+      p2 = __ldg(args.pos + 2 * N + tn);
+    }
+
+    for (int j0 = 0;;) {
 #pragma unroll
       for (int b = 0; b < kBatch; ++b) {
         if (ptr[b] != nullptr) {
@@ -148,6 +165,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
           __stcs(ptr[b] + half4, x2[b]);
         }
       }
+      j0 += kBatch;
+      if (j0 >= J) break;
+      load_batch(j0);
     }
   }
 }
