@@ -30,7 +30,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from vlm_decoder_positional_b200 import cmr, inputs  # noqa: E402
+from vlm_decoder_positional_b200 import cmr, inputs, shard  # noqa: E402
 
 METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/K, 1 GPU"
 UNIT = "tokens/s"
@@ -156,68 +156,82 @@ class ClockSampler:
 # CPU side: the oracle on a bounded sample (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl_cpu, n_seqs, n_tokens):
-    """One oracle pass over a sample: planes of the first n_seqs prompts, then
-    the rotation of their first n_tokens tokens, every layer and head."""
+def oracle_sample_step(wl_cpu, n):
+    """One oracle pass over a sample: the planes of the prompts that hold the
+    first n tokens (decode: of the first n prompts, then their new token),
+    then the rotation of those n tokens' Q/K rows, every layer and head."""
     import oracle
-    cu = wl_cpu["cu"][: n_seqs + 1]
-    ids = wl_cpu["ids"][: cu[-1]]
-    pos, _, _ = oracle.positions(ids, cu, inputs.IMAGE_TOKEN_ID)
-    p = np.ascontiguousarray(pos[:, :n_tokens])
-    oracle.rotate_bf16(wl_cpu["q"][:, :n_tokens], p)
-    oracle.rotate_bf16(wl_cpu["k"][:, :n_tokens], p)
-    return n_tokens
+    cu = wl_cpu["cu"]
+    if wl_cpu["cache_len"] is None:
+        b = int(np.searchsorted(cu, n, side="left"))
+        pos, _, _ = oracle.positions(wl_cpu["ids"][: cu[b]], cu[: b + 1], inputs.IMAGE_TOKEN_ID)
+        pos = np.ascontiguousarray(pos[:, :n])
+    else:
+        _, start, amount = oracle.positions(wl_cpu["ids"][: cu[n]], cu[: n + 1],
+                                            inputs.IMAGE_TOKEN_ID)
+        pos = oracle.positions_step(wl_cpu["cache_len"][:n], start, amount)
+    oracle.rotate_bf16(wl_cpu["q"][:, :n], pos)
+    oracle.rotate_bf16(wl_cpu["k"][:, :n], pos)
+    return n
 
 
-def cpu_sample_inputs(wl, n_tokens):
+def cpu_sample_inputs(wl, n_max):
     def bits(t):
-        return t[:, :n_tokens].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-    return {"ids": wl.ids, "cu": wl.cu_seqlens, "q": bits(wl.q), "k": bits(wl.k)}
+        return t[:, :n_max].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    return {"ids": wl.ids, "cu": wl.cu_seqlens, "q": bits(wl.q), "k": bits(wl.k),
+            "cache_len": wl.cache_len}
 
 
-def calibrate_sample(wl_cpu, seconds):
-    probe = 64
+def calibrate_sample(wl_cpu, seconds, n_max):
+    """Tokens whose oracle pass takes about `seconds` on this host (at most n_max)."""
+    probe = min(256, n_max)
     t0 = time.perf_counter()
-    oracle_sample_step(wl_cpu, 1, probe)
+    oracle_sample_step(wl_cpu, probe)
     dt = time.perf_counter() - t0
-    return int(max(probe, min(wl_cpu["q"].shape[1], probe * seconds / max(dt, 1e-6))))
+    return int(max(probe, min(n_max, probe * seconds / max(dt, 1e-6))))
+
+
+def sample_label(wl, n):
+    if wl.cache_len is not None:
+        return (f"planes of the first {n} prompts + their new token, rotation of those {n} "
+                f"tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
+    b = int(np.searchsorted(wl.cu_seqlens, n, side="left"))
+    return (f"planes of the first {b} prompts ({wl.cu_seqlens[b]} tokens) + rotation of the "
+            f"first {n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
 
 
 def run_cpu_baseline(wl, seconds):
-    cap = 8192
-    wl_cpu = cpu_sample_inputs(wl, cap)
-    n = calibrate_sample(wl_cpu, seconds)
-    n = min(n, cap)
+    # size the copy to the host from a quick estimate, then calibrate on it
+    n_max = min(wl.qk_tokens, 200_000)
+    wl_cpu = cpu_sample_inputs(wl, n_max)
+    n = calibrate_sample(wl_cpu, seconds, n_max)
     t0 = time.perf_counter()
-    oracle_sample_step(wl_cpu, 1, n)
+    oracle_sample_step(wl_cpu, n)
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"planes of prompt 0 ({wl.cu_seqlens[1]} tokens) + rotation of its first "
-                      f"{n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, "
-                      f"1 thread, {dt:.1f} s"}
+            "sample": sample_label(wl, n) + f", {dt:.1f} s"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    # the same prompts (ids); Q/K drawn only for the sampled first prompt
+    # the same prompts (ids); Q/K drawn only for the sampled tokens
     wl = inputs.make_config(args.workload, device="cpu", with_qk=False)
-    first = int(wl.cu_seqlens[1]) if wl.cache_len is None else wl.num_seqs
-    wl.q = inputs.random_qk((wl.num_layers, min(first, 8192), wl.hq, wl.head_dim), wl.seed + 1)
-    wl.k = inputs.random_qk((wl.num_layers, min(first, 8192), wl.hk, wl.head_dim), wl.seed + 2)
     per_step = max(1.0, args.reference_budget_s / (args.steps + args.warmup))
-    wl_cpu = cpu_sample_inputs(wl, 8192)
-    n = min(calibrate_sample(wl_cpu, per_step), 8192)
+    n_max = min(wl.num_seqs if wl.cache_len is not None else wl.n_tokens, 65_536)
+    wl.q = inputs.random_qk((wl.num_layers, n_max, wl.hq, wl.head_dim), wl.seed + 1)
+    wl.k = inputs.random_qk((wl.num_layers, n_max, wl.hk, wl.head_dim), wl.seed + 2)
+    wl_cpu = cpu_sample_inputs(wl, n_max)
+    n = calibrate_sample(wl_cpu, per_step, n_max)
     for _ in range(args.warmup):
-        oracle_sample_step(wl_cpu, 1, n)
+        oracle_sample_step(wl_cpu, n)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_sample_step(wl_cpu, 1, n)
+        oracle_sample_step(wl_cpu, n)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
-    sample = (f"per step: planes of prompt 0 ({wl.cu_seqlens[1]} tokens) + rotation of its "
-              f"first {n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
+    sample = "per step: " + sample_label(wl, n)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -252,9 +266,22 @@ def run_ours(args):
                                 device_id=dev)
     cmr.lib()
 
-    # weak scaling: every rank rotates its own batch (a different seed per rank)
-    wl = inputs.make_config(args.workload, device=dev,
-                            seed=inputs.BASE_SEED + args.workload + 1000 * rank)
+    if args.scaling == "weak":
+        # every rank rotates a full batch of its own (a different seed per rank)
+        wl = inputs.make_config(args.workload, device=dev,
+                                seed=shard.rank_seed(inputs.BASE_SEED + args.workload, rank))
+    else:
+        # one batch split by whole prompts; each rank draws only its own Q/K rows
+        wl = inputs.make_config(args.workload, device=dev, with_qk=False)
+        if wl.cache_len is not None:
+            raise SystemExit("--scaling strong covers prefill workloads only")
+        global_tokens = wl.n_tokens
+        sh = shard.shard_sequences(wl.cu_seqlens, world, rank)
+        wl.ids, wl.cu_seqlens = shard.local_batch(wl.ids, wl.cu_seqlens, sh)
+        wl.frame_origin = wl.frame_origin[sh.seq_lo:sh.seq_hi]
+        seed = shard.rank_seed(wl.seed, rank)
+        wl.q = inputs.random_qk((wl.num_layers, sh.n_tokens, wl.hq, wl.head_dim), seed + 1, dev)
+        wl.k = inputs.random_qk((wl.num_layers, sh.n_tokens, wl.hk, wl.head_dim), seed + 2, dev)
     ids = torch.from_numpy(wl.ids).to(dev)
     cu = torch.from_numpy(wl.cu_seqlens).to(dev)
     n, b, L = wl.n_tokens, wl.num_seqs, wl.num_layers
@@ -269,6 +296,8 @@ def run_ours(args):
     rot_b = rotate_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim)
 
     def step(ev=None):
+        if ev is not None:
+            ev[2].record(stream)
         p, s, a = cmr.positions(ids, cu, wl.image_token_id, out=(pos, start, amount))
         pr = cmr.positions_step(cache_len, s, a, out=pos_step) if decode else p
         if ev is not None:
@@ -281,7 +310,7 @@ def run_ours(args):
         step()
     torch.cuda.synchronize(dev)
 
-    rot_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    rot_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                   for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -297,34 +326,35 @@ def run_ours(args):
     if dist:
         dist.barrier()
     ms = t_begin.elapsed_time(t_end)
-    rot_ms = [a.elapsed_time(z) for a, z in rot_events]
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    rot_ms = [a.elapsed_time(z) for a, z, _ in rot_events]
+    pos_ms = [p.elapsed_time(a) for a, _, p in rot_events]
+    ms_max = shard.max_over_ranks(ms, dist, dev)
+    # tokens processed by all ranks in one step
+    tokens_all = tokens_per_step * world if args.scaling == "weak" else global_tokens
     launches = args.steps * (3 if decode else 2)
 
     # end to end through the public API from pinned host memory
-    e2e = run_e2e(args, wl, dev, stream, dist)
+    e2e = run_e2e(args, wl, dev, stream, dist, tokens_all)
 
     if rank == 0:
         peak, peak_src = measured_peak()
         rot_avg_s = statistics.mean(rot_ms) / 1e3
         achieved = rot_b / rot_avg_s / 1e9
         traffic = recorded_traffic(wl.name)
-        value = tokens_per_step * args.steps * world / (ms_max / 1e3)
+        value = tokens_all * args.steps / (ms_max / 1e3)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = run_cpu_baseline(wl, args.cpu_seconds)
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None,
+            "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 Q/K, uniform text ids, one 448x448 frame "
                     "per prompt)",
-            "config": {"workload": workload_label(wl), "global_batch": n * world,
-                       "seq_len": n // max(b, 1), "parallelism": f"dp{world} (independent "
-                       "batches, no data-path collective)",
+            "config": {"workload": workload_label(wl), "global_batch": tokens_all,
+                       "seq_len": n // max(b, 1),
+                       "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'whole prompts split over ranks'}, no data-path collective)",
                        "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
                              " no flush" % (rot_b / 1e9)},
             "hbm_gbs": achieved, "pct_of_peak": 100.0 * achieved / peak,
@@ -337,6 +367,7 @@ def run_ours(args):
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6650 GB/s"},
             "positions_bytes_per_step": positions_bytes(n, b),
+            "positions_avg_ms": statistics.mean(pos_ms),
             "e2e": e2e, "gpu_launches": launches, "clocks": clocks.summary(),
             "cpu_baseline": cpu, "impl": "ours",
         }
@@ -347,7 +378,7 @@ def run_ours(args):
     return 0
 
 
-def run_e2e(args, wl, dev, stream, dist):
+def run_e2e(args, wl, dev, stream, dist, tokens_all):
     """Same metric through the public API: every step copies the inputs from
     pinned host memory, runs positions + rotate, and reads the results back."""
     steps = max(2, min(args.steps, args.e2e_steps))
@@ -389,16 +420,13 @@ def run_e2e(args, wl, dev, stream, dist):
         step()
     z.record(stream)
     torch.cuda.synchronize(dev)
-    ms = torch.tensor([a.elapsed_time(z)], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    world = dist.get_world_size() if dist else 1
+    ms = shard.max_over_ranks(a.elapsed_time(z), dist, dev)
     h2d = (h_ids.numel() * 4 + h_cu.numel() * 4 + h_q.numel() * 2 + h_k.numel() * 2
            + (h_cl.numel() * 4 if decode else 0))
     d2h = h_q.numel() * 2 + h_k.numel() * 2 + h_pos.numel() * 4 + 8 * wl.num_seqs
-    return {"value": wl.qk_tokens * steps * world / (float(ms.item()) / 1e3), "unit": UNIT,
+    return {"value": tokens_all * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "ms_per_step": float(ms.item()) / steps,
+            "ms_per_step": ms / steps,
             "path": "pinned host -> cmr.positions + cmr.rotate_qk -> pinned host"}
 
 
@@ -411,6 +439,9 @@ def main():
     ap.add_argument("--workload", type=int, default=5, choices=[1, 2, 3, 4, 5],
                     help="1..5: single 80-token prompt, varlen 16, 64x4096 outliers, "
                          "decode 1024, 6 layers x 32 x 8192 (default)")
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="weak: a full batch per GPU (default); strong: one batch split by "
+                         "whole prompts")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)

@@ -13,9 +13,12 @@
  *   [P2] Hugging Face card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, section
  *        "How the VLM rides the text-only engine" (engine I/O table and the
  *        canvas table), and "What it is" (interleaved sections [11, 11, 10]).
- * The rotation's open parameters (rotate-half on the first rot_dim dims,
- * inv_freq = theta^(-2j/rot_dim), theta = 1e7, the interleave map) are the
- * readings fixed by the workload specification and listed in the design doc.
+ * The pages do not print the rotation's own parameters.  The oracle takes the
+ * reading fixed for this model: rotate-half on the first rot_dim (64) dims of
+ * each 256-dim head, pairs (d, d + rot_dim/2), one frequency per pair with
+ * inv_freq = theta^(-2j/rot_dim), theta = 1e7, and the interleave that gives
+ * frequency j to H when j % 3 == 1 and j < 33, to W when j % 3 == 2 and
+ * j < 30, and to T otherwise.
  *
  * Every loop follows the rule in the pages' order; there is no blocking,
  * fusion or reordering.  Pins for every function live in tests/ (-m "not gpu").

@@ -8,7 +8,8 @@
 // Work split: CTA (b, s) owns slice s of prompt b.  To know the origin O it
 // scans the prompt's ids from index 0 up to the end of its own slice (slice 0
 // scans the whole prompt, since it also writes start/amount), in chunks of
-// 2048 ids, and stops at the first chunk that holds a marker.  A marker past
+// 8192 ids (16 loads in flight per thread), and stops at the first chunk that
+// holds a marker.  A marker past
 // the slice cannot change the slice's planes (every token there is p < O ->
 // (p, p, p), the same as text-only), so no CTA waits on another and there is
 // no scratch memory and no atomics.  Ids re-read by later slices hit L2.
@@ -19,9 +20,9 @@
 namespace cmr {
 namespace {
 
-constexpr int kPosThreads = 256;
-constexpr int kIdsPerThread = 8;
-constexpr int kScanChunk = kPosThreads * kIdsPerThread;  // 2048 ids per step
+constexpr int kPosThreads = 512;
+constexpr int kIdsPerThread = 16;
+constexpr int kScanChunk = kPosThreads * kIdsPerThread;  // 8192 ids per step
 constexpr int kSliceTarget = 2048;                       // tokens per CTA (target)
 constexpr int kMaxSlices = 65535;                        // gridDim.y limit
 
