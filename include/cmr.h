@@ -53,6 +53,11 @@ typedef enum cmr_status {
 /* Bits a kernel ORs into the optional device status word. */
 #define CMR_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens not 0 .. n_tokens, non-decreasing */
 
+/* Position rules for cmr_positions_chunk. */
+#define CMR_RULE_CANVAS 0    /* this model's canvas rule: start = O + 67, amount 58 */
+#define CMR_RULE_QWEN_VL 1   /* Qwen-VL's shift: start = O + 65, amount 56 */
+#define CMR_RULE_PLANES_1D 2 /* plain 1-D positions: (p, p, p), state (2^30, 0) */
+
 /* Planes of a packed batch of prompts (the canvas table, HF card
  * mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides the text-only
  * engine").  For prompt b, O = the first local index whose id equals
@@ -88,6 +93,45 @@ CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
                          int32_t image_token_id, int32_t* out_pos,
                          int32_t* out_start, int32_t* out_amount,
                          int32_t* device_status, cmr_stream_t stream);
+
+/* Planes of a batch of prompt CHUNKS: chunked prefill, and later turns that
+ * append to a kept state (port notes, "Prefill in chunks and a second turn":
+ * S = 16 prefill answers as the one-token order; a second question reuses
+ * the state after turn 1).  Chunk b is ids[cu[b] .. cu[b+1]) and holds the
+ * absolute indices pos_offset[b] + 0, 1, ... of its sequence.  The sequence's
+ * state before the chunk is (in_start[b], in_amount[b]) -- (2^30, 0) while no
+ * <image> has been seen, the value cmr_positions / an earlier chunk returned
+ * otherwise.  If a frame is known, its origin follows from amount = start -
+ * (O + 9); if not, the chunk's first marker at local index m sets O =
+ * pos_offset[b] + m and
+ *   CMR_RULE_CANVAS:    start = O + 67, amount = 58 (as cmr_positions);
+ *   CMR_RULE_QWEN_VL:   start = O + 65, amount = 56 (port notes, CoreAIKit:
+ *                       Qwen-VL's rule "would give + 64 and 56" from the
+ *                       pads; </image> and "\n" then count as text after the
+ *                       frame);
+ *   CMR_RULE_PLANES_1D: no shift at all, state (2^30, 0) (the LiteRT card:
+ *                       the runtime feeds plain 1-D positions).
+ * Each token gets the canvas table's row at its absolute index.  With all
+ * offsets 0, no incoming state and CMR_RULE_CANVAS this is cmr_positions.
+ *
+ *   ids, cu_seqlens, num_seqs, n_tokens, image_token_id, out_pos,
+ *   device_status   as in cmr_positions
+ *   rule            one of CMR_RULE_*
+ *   pos_offset      device int32 [num_seqs], or NULL for all zeros
+ *   in_start, in_amount   device int32 [num_seqs], or NULL for (2^30, 0)
+ *   out_start, out_amount device int32 [num_seqs]: the state after the chunk.
+ *                   Must not overlap in_start / in_amount (use two buffers and
+ *                   swap them between chunks).
+ * Errors: as cmr_positions, plus CMR_EINVAL for an unknown rule or
+ * overlapping incoming and outgoing state. */
+CMR_API cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens,
+                                       int32_t num_seqs, int64_t n_tokens,
+                                       int32_t image_token_id, int32_t rule,
+                                       const int32_t* pos_offset,
+                                       const int32_t* in_start,
+                                       const int32_t* in_amount, int32_t* out_pos,
+                                       int32_t* out_start, int32_t* out_amount,
+                                       int32_t* device_status, cmr_stream_t stream);
 
 /* Planes of one new token per sequence, for decode and continuation (port
  * notes: "every generated token at p - amount"; canvas table row "everything
@@ -138,6 +182,31 @@ CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n
                          int32_t head_dim, double theta,
                          const int32_t sections[3], int32_t rot_dim,
                          cmr_stream_t stream);
+
+/* cmr_rotate_qk with the planes derived inside the kernel instead of read
+ * from pos [3, n_tokens]: token t of prompt b (cu[b] <= t < cu[b+1]) sits at
+ * absolute index p = pos_offset[b] + t - cu[b] and gets the canvas table's
+ * row for p under its sequence's (start[b], amount[b]), exactly as
+ * cmr_positions_step would give it.  One launch then covers a decode step
+ * (cu_seqlens = NULL: token b is sequence b, p = pos_offset[b]) or a prefill
+ * chunk whose state is known, and the 24 B/token pos round trip disappears.
+ *
+ *   q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections, rot_dim
+ *                 as in cmr_rotate_qk
+ *   cu_seqlens    device int32 [num_seqs + 1] as in cmr_positions (it must be
+ *                 well formed: it is not checked on the device), or NULL when
+ *                 num_seqs == n_tokens and each sequence holds one token
+ *   pos_offset    device int32 [num_seqs], or NULL for all zeros
+ *   start, amount device int32 [num_seqs]
+ * Errors: as cmr_rotate_qk, plus CMR_EINVAL for num_seqs <= 0 with tokens,
+ * missing start/amount, or cu_seqlens == NULL with num_seqs != n_tokens. */
+CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens,
+                                       int32_t num_seqs, const int32_t* pos_offset,
+                                       const int32_t* start, const int32_t* amount,
+                                       int64_t n_tokens, int32_t num_layers, int32_t hq,
+                                       int32_t hk, int32_t head_dim, double theta,
+                                       const int32_t sections[3], int32_t rot_dim,
+                                       cmr_stream_t stream);
 
 /* Static, never-null description of a status code. */
 CMR_API const char* cmr_status_string(cmr_status s);

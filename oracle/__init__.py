@@ -25,6 +25,8 @@ RULE_AMOUNT_PLUS_ONE = 1
 RULE_PLANES_1D = 2
 _RULES = {"canvas": RULE_CANVAS, "amount+1": RULE_AMOUNT_PLUS_ONE,
           "planes_1d": RULE_PLANES_1D}
+CHUNK_RULES = {"canvas": 0, "qwen_vl": 1, "planes_1d": 2}
+TEXT_ONLY_START = 1 << 30
 
 _lib = None
 
@@ -37,6 +39,10 @@ def _load():
         lib.oracle_positions.argtypes = [i32p, i32p, ctypes.c_int32, ctypes.c_int64,
                                          ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p]
         lib.oracle_positions.restype = ctypes.c_int
+        lib.oracle_positions_chunk.argtypes = [i32p, i32p, ctypes.c_int32, ctypes.c_int64,
+                                               ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p,
+                                               i32p, i32p, i32p]
+        lib.oracle_positions_chunk.restype = ctypes.c_int
         lib.oracle_positions_step.argtypes = [i32p, i32p, i32p, ctypes.c_int32, i32p]
         lib.oracle_positions_step.restype = ctypes.c_int
         lib.oracle_freq_planes.argtypes = [ctypes.c_int32, i32p, i32p]
@@ -81,6 +87,35 @@ def positions(ids, cu_seqlens, image_token_id=248078, rule="canvas"):
                               _i32(pos)[1], _i32(start)[1], _i32(amount)[1])
     if st != 0:
         raise OracleError("oracle_positions: invalid arguments")
+    return pos, start, amount
+
+
+def positions_chunk(ids, cu_seqlens, image_token_id=248078, rule="canvas", pos_offset=None,
+                    in_start=None, in_amount=None):
+    """Planes of a batch of prompt chunks at absolute offsets, continuing each
+    sequence's (start, amount) state.  Returns (pos [3, N], start [B], amount [B])."""
+    lib = _load()
+    ids, ids_p = _i32(ids)
+    cu, cu_p = _i32(cu_seqlens)
+    n = int(ids.shape[0])
+    b = int(cu.shape[0]) - 1
+    opt = []
+    for a in (pos_offset, in_start, in_amount):
+        if a is None:
+            opt.append((None, None))
+        else:
+            arr, ptr = _i32(a)
+            if arr.shape[0] != b:
+                raise OracleError("per-sequence arrays need num_seqs entries")
+            opt.append((arr, ptr))
+    pos = np.zeros((3, n), dtype=np.int32)
+    start = np.zeros(max(b, 0), dtype=np.int32)
+    amount = np.zeros(max(b, 0), dtype=np.int32)
+    st = lib.oracle_positions_chunk(ids_p, cu_p, b, n, int(image_token_id), CHUNK_RULES[rule],
+                                    opt[0][1], opt[1][1], opt[2][1], _i32(pos)[1],
+                                    _i32(start)[1], _i32(amount)[1])
+    if st != 0:
+        raise OracleError("oracle_positions_chunk: invalid arguments")
     return pos, start, amount
 
 

@@ -152,6 +152,76 @@ int oracle_positions(const int32_t* ids, const int32_t* cu_seqlens,
   return ORC_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Chunks of prompts: chunked prefill and later turns                         */
+/* ------------------------------------------------------------------------ */
+
+/* Rules for the chunked form: the canvas rule; Qwen-VL's shift, which the
+ * port notes' CoreAIKit section gives as "+ 64 and 56" from the index where the
+ * pads begin (start = O + 65, so </image> and "\n" count as text after the
+ * frame, amount = start - (O + 9) = 56); and plain 1-D positions (the LiteRT
+ * card: the runtime feeds plain 1-D positions). */
+#define CHUNK_RULE_CANVAS 0
+#define CHUNK_RULE_QWEN_VL 1
+#define CHUNK_RULE_PLANES_1D 2
+#define QWEN_VL_FRAME_SHIFT 65
+
+/* Chunk b holds the absolute indices pos_offset[b] + [0, len_b) of its
+ * sequence (a prefill chunk, or the next turn appended to a kept state).
+ * in_start / in_amount (either may be NULL: no state yet) carry what earlier
+ * chunks established: (2^30, 0) while no <image> has been seen, else the
+ * sequence's start and amount.  With a frame already seen, its origin follows
+ * from amount = start - (O + 9).  Otherwise the chunk's first marker, if any,
+ * sets O (absolute) and start / amount by the rule.  Every token then gets the
+ * canvas table's row at its absolute index.  out_start / out_amount receive
+ * the sequence's state after the chunk. */
+int oracle_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens,
+                           int32_t num_seqs, int64_t n_tokens,
+                           int32_t image_token_id, int32_t rule,
+                           const int32_t* pos_offset, const int32_t* in_start,
+                           const int32_t* in_amount, int32_t* pos,
+                           int32_t* start_out, int32_t* amount_out) {
+  if (num_seqs < 0 || n_tokens < 0) return ORC_EINVAL;
+  if (rule < CHUNK_RULE_CANVAS || rule > CHUNK_RULE_PLANES_1D) return ORC_EINVAL;
+  if (num_seqs == 0) return n_tokens == 0 ? ORC_OK : ORC_EINVAL;
+  if (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[num_seqs] != n_tokens)
+    return ORC_EINVAL;
+  for (int32_t b = 0; b < num_seqs; ++b)
+    if (cu_seqlens[b + 1] < cu_seqlens[b]) return ORC_EINVAL;
+
+  for (int32_t b = 0; b < num_seqs; ++b) {
+    const int64_t first = cu_seqlens[b];
+    const int64_t len = (int64_t)cu_seqlens[b + 1] - first;
+    const int64_t offset = pos_offset ? pos_offset[b] : 0;
+    int64_t start = in_start ? in_start[b] : TEXT_ONLY_START;
+    int64_t amount = in_amount ? in_amount[b] : 0;
+
+    if (rule == CHUNK_RULE_PLANES_1D) {
+      start = TEXT_ONLY_START;
+      amount = 0;
+    } else if (start >= TEXT_ONLY_START) {
+      /* no frame yet: the chunk's first <image>, if any, is the origin */
+      for (int64_t p = 0; p < len; ++p) {
+        if (ids[first + p] == image_token_id) {
+          const int64_t O = offset + p;
+          start = O + (rule == CHUNK_RULE_QWEN_VL ? QWEN_VL_FRAME_SHIFT : FRAME_TOKENS);
+          amount = start - (O + CANVAS_SPAN);
+          break;
+        }
+      }
+    }
+    start_out[b] = (int32_t)start;
+    amount_out[b] = (int32_t)amount;
+
+    for (int64_t p = 0; p < len; ++p) {
+      int64_t v[3];
+      planes_from_shift(offset + p, start, amount, v);
+      for (int r = 0; r < 3; ++r) pos[r * n_tokens + first + p] = (int32_t)v[r];
+    }
+  }
+  return ORC_OK;
+}
+
 /* Decode / continuation: the token at absolute index p = cache_len[b] of
  * sequence b, with that sequence's start and amount.  Generated tokens sit at
  * p - amount on all three planes ([P1] "every generated token at p - amount";

@@ -27,8 +27,9 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    assert set(names) == {"cmr_positions", "cmr_positions_step", "cmr_rotate_qk",
-                          "cmr_status_string", "cmr_last_error_message", "cmr_version"}
+    assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
+                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_status_string",
+                          "cmr_last_error_message", "cmr_version"}
     assert set(names) == set(cmr.SIGNATURES)
 
 
@@ -47,7 +48,7 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 10000
+    assert lib.cmr_version() == 10100
 
 
 SEC = (ctypes.c_int32 * 3)(11, 11, 10)
@@ -96,3 +97,31 @@ def test_positions_empty_batch_is_a_no_op(lib):
     assert lib.cmr_positions(None, None, 0, 0, 248078, None, None, None, None, None) == 0
     assert lib.cmr_positions_step(None, None, None, 0, None, None) == 0
     assert lib.cmr_positions_step(None, None, None, -1, None, None) == cmr.CMR_EINVAL
+
+
+@pytest.mark.parametrize("kw", [
+    dict(rule=3), dict(rule=-1), dict(num_seqs=-1), dict(cu=None),
+    dict(in_start=FAKE + 64, out_start=FAKE + 64), dict(in_amount=FAKE + 64, out_start=FAKE + 64),
+    dict(in_start=FAKE + 60, out_amount=FAKE + 64),
+])
+def test_positions_chunk_rejects_bad_arguments_on_the_host(lib, kw):
+    a = dict(ids=FAKE, cu=FAKE, num_seqs=2, n=10, rule=0, off=None, in_start=FAKE + 256,
+             in_amount=FAKE + 512, pos=FAKE, out_start=FAKE + 1024, out_amount=FAKE + 2048)
+    a.update(kw)
+    st = lib.cmr_positions_chunk(a["ids"], a["cu"], a["num_seqs"], a["n"], 248078, a["rule"],
+                                 a["off"], a["in_start"], a["in_amount"], a["pos"],
+                                 a["out_start"], a["out_amount"], None, None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+
+
+@pytest.mark.parametrize("kw", [
+    dict(num_seqs=0), dict(start=None), dict(amount=None), dict(cu=None, num_seqs=3),
+    dict(rot_dim=24), dict(q=FAKE + 4),
+])
+def test_rotate_shift_rejects_bad_arguments_on_the_host(lib, kw):
+    a = dict(q=FAKE, k=FAKE, cu=FAKE, num_seqs=2, off=None, start=FAKE, amount=FAKE, n=10,
+             rot_dim=64)
+    a.update(kw)
+    st = lib.cmr_rotate_qk_shift(a["q"], a["k"], a["cu"], a["num_seqs"], a["off"], a["start"],
+                                 a["amount"], a["n"], 1, 8, 2, 256, 1e7, SEC, a["rot_dim"], None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()

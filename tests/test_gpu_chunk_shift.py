@@ -1,0 +1,163 @@
+"""GPU parity of the chunked positions form, its rules, and the rotate that
+derives the planes in the kernel, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import assert_bf16_close
+from vlm_decoder_positional_b200 import cmr, inputs
+
+pytestmark = pytest.mark.gpu
+MARK = inputs.IMAGE_TOKEN_ID
+
+
+def t32(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+
+
+def bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def chunk_batches(wl, size):
+    """Split every prompt of a workload into consecutive chunks of `size`
+    tokens; step i holds the i-th chunk of every prompt (empty once done)."""
+    lens = np.diff(wl.cu_seqlens)
+    steps = int(np.ceil(lens.max() / size))
+    for i in range(steps):
+        lo = np.minimum(lens, i * size)
+        hi = np.minimum(lens, (i + 1) * size)
+        parts = [wl.ids[wl.cu_seqlens[b] + lo[b]: wl.cu_seqlens[b] + hi[b]]
+                 for b in range(wl.num_seqs)]
+        ids, cu = inputs.pack(parts)
+        yield ids, cu, lo.astype(np.int32)
+
+
+@pytest.mark.parametrize("cfg,size", [(1, 16), (2, 16), (2, 100), (3, 1000), (5, 4096)])
+@pytest.mark.parametrize("rule", ["canvas", "qwen_vl", "planes_1d"])
+def test_chunked_prefill_bit_exact(cuda_device, cfg, size, rule):
+    wl = inputs.make_config(cfg, with_qk=False)
+    dev = cuda_device
+    b = wl.num_seqs
+    g_state = (t32(np.full(b, 1 << 30), dev), t32(np.zeros(b), dev))
+    o_state = (np.full(b, 1 << 30, np.int32), np.zeros(b, np.int32))
+    got_all, want_all = [], []
+    for ids, cu, off in chunk_batches(wl, size):
+        g_out = (torch.empty((3, ids.size), dtype=torch.int32, device=dev),
+                 torch.empty(b, dtype=torch.int32, device=dev),
+                 torch.empty(b, dtype=torch.int32, device=dev))
+        pos, s, a = cmr.positions_chunk(t32(ids, dev), t32(cu, dev), t32(off, dev), g_state,
+                                        rule, out=g_out)
+        wpos, ws, wa = oracle.positions_chunk(ids, cu, MARK, rule, off, *o_state)
+        np.testing.assert_array_equal(pos.cpu().numpy(), wpos)
+        np.testing.assert_array_equal(s.cpu().numpy(), ws)
+        np.testing.assert_array_equal(a.cpu().numpy(), wa)
+        g_state, o_state = (s, a), (ws, wa)
+        got_all.append(pos.cpu().numpy())
+    if rule == "canvas":
+        # the chunks together give the whole-prompt planes
+        whole = oracle.positions(wl.ids, wl.cu_seqlens, MARK)[0]
+        per_prompt = {b_: [] for b_ in range(b)}
+        for (ids, cu, off), pos in zip(chunk_batches(wl, size), got_all):
+            for b_ in range(b):
+                per_prompt[b_].append(pos[:, cu[b_]:cu[b_ + 1]])
+        for b_ in range(b):
+            np.testing.assert_array_equal(np.concatenate(per_prompt[b_], axis=1),
+                                          whole[:, wl.cu_seqlens[b_]:wl.cu_seqlens[b_ + 1]])
+
+
+def test_rules_on_whole_prompts(cuda_device):
+    for cfg in (2, 3):
+        wl = inputs.make_config(cfg, with_qk=False)
+        for rule in ("canvas", "qwen_vl", "planes_1d"):
+            pos, s, a = cmr.positions_chunk(t32(wl.ids, cuda_device), t32(wl.cu_seqlens, cuda_device),
+                                            rule=rule)
+            wpos, ws, wa = oracle.positions_chunk(wl.ids, wl.cu_seqlens, MARK, rule)
+            np.testing.assert_array_equal(pos.cpu().numpy(), wpos)
+            np.testing.assert_array_equal(s.cpu().numpy(), ws)
+            np.testing.assert_array_equal(a.cpu().numpy(), wa)
+
+
+def test_overlapping_state_is_rejected(cuda_device):
+    ids = t32(np.zeros(8), cuda_device)
+    cu = t32([0, 8], cuda_device)
+    st = t32([1 << 30], cuda_device)
+    am = t32([0], cuda_device)
+    with pytest.raises(cmr.CmrError):
+        cmr.positions_chunk(ids, cu, state=(st, am),
+                            out=(torch.empty((3, 8), dtype=torch.int32, device=cuda_device), st, am))
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 5])
+def test_shift_rotate_equals_pos_rotate_bit_for_bit(cuda_device, cfg):
+    wl = inputs.make_config(cfg, device=cuda_device)
+    dev = cuda_device
+    ids, cu = t32(wl.ids, dev), t32(wl.cu_seqlens, dev)
+    pos, s, a = cmr.positions(ids, cu)
+    q2, k2 = wl.q.clone(), wl.k.clone()
+    cmr.rotate_qk(wl.q, wl.k, pos)
+    cmr.rotate_qk_shift(q2, k2, s, a, cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert torch.equal(wl.q.view(torch.int16), q2.view(torch.int16))
+    assert torch.equal(wl.k.view(torch.int16), k2.view(torch.int16))
+
+
+def test_decode_step_in_one_launch(cuda_device):
+    wl = inputs.make_config(4, device=cuda_device)
+    dev = cuda_device
+    _, s, a = cmr.positions(t32(wl.ids, dev), t32(wl.cu_seqlens, dev))
+    cache_len = t32(wl.cache_len, dev)
+    q_in, k_in = bits(wl.q), bits(wl.k)
+    q2, k2 = wl.q.clone(), wl.k.clone()
+    cmr.rotate_qk_shift(wl.q, wl.k, s, a, pos_offset=cache_len)          # one launch
+    cmr.rotate_qk(q2, k2, cmr.positions_step(cache_len, s, a))           # two launches
+    torch.cuda.synchronize()
+    assert torch.equal(wl.q.view(torch.int16), q2.view(torch.int16))
+    p = oracle.positions_step(wl.cache_len, s.cpu().numpy(), a.cpu().numpy())
+    assert_bf16_close(bits(wl.q), oracle.rotate_bf16(q_in, p), "decode q")
+    assert_bf16_close(bits(wl.k), oracle.rotate_bf16(k_in, p), "decode k")
+
+
+def test_shift_rotate_on_chunks_at_offsets(cuda_device):
+    # the second chunk of every prompt of the varlen workload, rotated with the
+    # state the first chunk left
+    wl = inputs.make_config(2, device=cuda_device)
+    dev = cuda_device
+    first = [wl.ids[wl.cu_seqlens[b]: wl.cu_seqlens[b] + 60] for b in range(wl.num_seqs)]
+    rest = [wl.ids[wl.cu_seqlens[b] + 60: wl.cu_seqlens[b + 1]] for b in range(wl.num_seqs)]
+    ids1, cu1 = inputs.pack(first)
+    ids2, cu2 = inputs.pack(rest)
+    _, s, a = cmr.positions_chunk(t32(ids1, dev), t32(cu1, dev))
+    off = t32(np.full(wl.num_seqs, 60), dev)
+    n2 = ids2.size
+    g = torch.Generator(device=dev).manual_seed(9)
+    q = torch.randn((1, n2, 8, 256), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((1, n2, 2, 256), generator=g, device=dev).to(torch.bfloat16)
+    q_in, k_in = bits(q), bits(k)
+    cmr.rotate_qk_shift(q, k, s, a, cu_seqlens=t32(cu2, dev), pos_offset=off)
+    torch.cuda.synchronize()
+    whole = oracle.positions(wl.ids, wl.cu_seqlens, MARK)[0]
+    p = np.concatenate([whole[:, wl.cu_seqlens[b] + 60: wl.cu_seqlens[b + 1]]
+                        for b in range(wl.num_seqs)], axis=1)
+    assert_bf16_close(bits(q), oracle.rotate_bf16(q_in, p), "chunk q")
+    assert_bf16_close(bits(k), oracle.rotate_bf16(k_in, p), "chunk k")
+
+
+def test_shift_rotate_with_empty_prompts(cuda_device):
+    rng = np.random.default_rng(6)
+    lens, origins = [0, 5, 0, 0, 90, 1, 0], [-1, 1, -1, -1, 20, 0, -1]
+    prompts = [inputs.prompt_ids(rng, n, o) for n, o in zip(lens, origins)]
+    ids, cu = inputs.pack(prompts)
+    dev = cuda_device
+    pos, s, a = cmr.positions(t32(ids, dev), t32(cu, dev))
+    n = ids.size
+    g = torch.Generator(device=dev).manual_seed(2)
+    q = torch.randn((3, n, 8, 256), generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn((3, n, 2, 256), generator=g, device=dev).to(torch.bfloat16)
+    q2, k2 = q.clone(), k.clone()
+    cmr.rotate_qk(q, k, pos)
+    cmr.rotate_qk_shift(q2, k2, s, a, cu_seqlens=t32(cu, dev))
+    torch.cuda.synchronize()
+    assert torch.equal(q.view(torch.int16), q2.view(torch.int16))
+    assert torch.equal(k.view(torch.int16), k2.view(torch.int16))

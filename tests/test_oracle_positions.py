@@ -210,3 +210,102 @@ def test_decode_config_positions():
     assert (amount == 58).all() and (start == wl.frame_origin + 67).all()
     step = oracle.positions_step(wl.cache_len, start, amount)
     assert (step == wl.cache_len - 58).all()
+
+
+# ---------------------------------------------------------------------------
+# chunked prefill, later turns and the rule variants
+# ---------------------------------------------------------------------------
+
+def run_in_chunks(ids, cuts, rule="canvas"):
+    """Feed one prompt to the chunked form in pieces, carrying the state."""
+    start = np.array([oracle.TEXT_ONLY_START], np.int32)
+    amount = np.array([0], np.int32)
+    out = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        pos, start, amount = oracle.positions_chunk(ids[lo:hi], np.array([0, hi - lo], np.int32),
+                                                    MARK, rule, np.array([lo], np.int32),
+                                                    start, amount)
+        out.append(pos)
+    return np.concatenate(out, axis=1), int(start[0]), int(amount[0])
+
+
+@pytest.mark.parametrize("O", [-1, 0, 6, 17, 40, 100])
+@pytest.mark.parametrize("chunk", [1, 16, 23, 67, 1000])
+def test_chunked_prefill_reproduces_the_whole_prompt(O, chunk):
+    # The port notes' S = 16 prefill answers as the one-token order: splitting
+    # a prompt anywhere (inside the frame too) must not change a plane.
+    ids, cu = one_prompt(300, O)
+    whole, start, amount = oracle.positions(ids, cu, MARK)
+    cuts = list(range(0, 300, chunk)) + [300]
+    got, s, a = run_in_chunks(ids, cuts)
+    np.testing.assert_array_equal(got, whole)
+    assert (s, a) == (int(start[0]), int(amount[0]))
+
+
+def test_second_turn_continues_the_kept_state():
+    # A second question on the same image: turn 2's ids are appended to turn 1's
+    # conversation and prefilled from the kept state (port notes, "Prefill in
+    # chunks and a second turn"); the planes equal those of the whole conversation.
+    rng = np.random.default_rng(21)
+    turn1 = inputs.prompt_ids(rng, 88, 6)
+    answer = inputs.text_ids(rng, 33)
+    turn2 = inputs.text_ids(rng, 20)
+    conv = np.concatenate([turn1, answer, turn2])
+    whole, _, _ = oracle.positions(conv, np.array([0, conv.size], np.int32), MARK)
+    got, s, a = run_in_chunks(conv, [0, 88, 121, conv.size])
+    np.testing.assert_array_equal(got, whole)
+    assert (s, a) == (73, 58)
+    assert whole[:, -1].tolist() == [conv.size - 1 - 58] * 3
+
+
+def test_chunked_batch_matches_per_sequence_chunks():
+    rng = np.random.default_rng(22)
+    n_seq = 7
+    prompts = [inputs.prompt_ids(rng, 200, o) for o in (3, -1, 0, 50, 120, 190, -1)]
+    offsets = np.array([0, 0, 17, 40, 100, 150, 199], np.int32)
+    states = []
+    for p, off in zip(prompts, offsets):
+        _, s, a = oracle.positions_chunk(p[:off], np.array([0, off], np.int32), MARK)
+        states.append((s[0], a[0]))
+    tails = [p[off:] for p, off in zip(prompts, offsets)]
+    ids, cu = inputs.pack(tails)
+    st = np.array([s for s, _ in states], np.int32)
+    am = np.array([a for _, a in states], np.int32)
+    pos, s_out, a_out = oracle.positions_chunk(ids, cu, MARK, "canvas", offsets, st, am)
+    for b in range(n_seq):
+        whole, ws, wa = oracle.positions(prompts[b], np.array([0, 200], np.int32), MARK)
+        np.testing.assert_array_equal(pos[:, cu[b]:cu[b + 1]], whole[:, offsets[b]:])
+        assert (s_out[b], a_out[b]) == (ws[0], wa[0])
+
+
+def test_qwen_vl_rule_shift_values():
+    # CoreAIKit section of the port notes: the canvas shifts from where the pads
+    # begin + 66 by 58; Qwen-VL's rule would give + 64 and 56.
+    for O in (6, 17):
+        ids, cu = one_prompt(O + 120, O)
+        pads_begin = O + 1
+        _, s, a = oracle.positions_chunk(ids, cu, MARK, "canvas")
+        assert (int(s[0]), int(a[0])) == (pads_begin + 66, 58)
+        pos, s, a = oracle.positions_chunk(ids, cu, MARK, "qwen_vl")
+        assert (int(s[0]), int(a[0])) == (pads_begin + 64, 56)
+        # </image> and "\n" now count as text after the frame, which resumes at O + 9
+        assert pos[:, O + 65].tolist() == [O + 9] * 3
+        assert pos[:, O + 66].tolist() == [O + 10] * 3
+        canvas, _, _ = oracle.positions(ids, cu, MARK)
+        np.testing.assert_array_equal(pos[:, :O + 65], canvas[:, :O + 65])
+
+
+def test_planes_1d_rule_is_plain_positions():
+    ids, cu = one_prompt(150, 10)
+    pos, s, a = oracle.positions_chunk(ids, cu, MARK, "planes_1d", np.array([1000], np.int32))
+    assert (int(s[0]), int(a[0])) == (2 ** 30, 0)
+    for r in range(3):
+        np.testing.assert_array_equal(pos[r], 1000 + np.arange(150))
+
+
+def test_chunk_form_at_offset_zero_is_the_prompt_form():
+    wl = inputs.make_config(2, with_qk=False)
+    a = oracle.positions(wl.ids, wl.cu_seqlens, MARK)
+    b = oracle.positions_chunk(wl.ids, wl.cu_seqlens, MARK)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)

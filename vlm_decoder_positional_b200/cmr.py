@@ -16,6 +16,8 @@ LIB_PATH = os.path.join(_PKG, "libcmr.so")
 
 CMR_OK, CMR_EINVAL, CMR_ECUDA, CMR_EUNSUPPORTED = 0, 1, 2, 3
 CMR_DEVICE_BAD_CU_SEQLENS = 1
+RULES = {"canvas": 0, "qwen_vl": 1, "planes_1d": 2}
+TEXT_ONLY_START = 1 << 30
 
 IMAGE_TOKEN_ID = 248078
 
@@ -24,8 +26,17 @@ _i32p = ctypes.c_void_p
 SIGNATURES = {
     "cmr_positions": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
                                      _i32p, _i32p, _i32p, _i32p, ctypes.c_void_p]),
+    "cmr_positions_chunk": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                           ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
+                                           _i32p, _i32p, _i32p, _i32p, ctypes.c_void_p]),
     "cmr_positions_step": (ctypes.c_int, [_i32p, _i32p, _i32p, ctypes.c_int32, _i32p,
                                           ctypes.c_void_p]),
+    "cmr_rotate_qk_shift": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p,
+                                           ctypes.c_int32, _i32p, _i32p, _i32p, ctypes.c_int64,
+                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_double,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                           ctypes.c_void_p]),
     "cmr_rotate_qk": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p, ctypes.c_int64,
                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.c_double,
@@ -124,6 +135,60 @@ def positions(ids: torch.Tensor, cu_seqlens: torch.Tensor, image_token_id: int =
     return pos, start, amount
 
 
+def positions_chunk(ids: torch.Tensor, cu_seqlens: torch.Tensor,
+                    pos_offset: Optional[torch.Tensor] = None,
+                    state: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                    rule: str = "canvas", image_token_id: int = IMAGE_TOKEN_ID,
+                    out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                    device_status: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """cmr_positions_chunk: planes of prompt chunks at absolute offsets, carrying
+    each sequence's (start, amount) state.  Returns (pos [3, N], start [B],
+    amount [B]) -- the state after the chunk."""
+    _want(ids, "ids", torch.int32)
+    dev = ids.device
+    _want(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    n, b = ids.numel(), cu_seqlens.numel() - 1
+    if b < 0:
+        raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+    if rule not in RULES:
+        raise ValueError(f"rule must be one of {sorted(RULES)}")
+    per_seq = [(pos_offset, "pos_offset")]
+    if state is not None:
+        per_seq += [(state[0], "in_start"), (state[1], "in_amount")]
+    for t, name in per_seq:
+        if t is None:
+            continue
+        _want(t, name, torch.int32, dev)
+        if t.numel() != b:
+            raise ValueError(f"{name} needs num_seqs entries")
+    off_ptr = pos_offset.data_ptr() if pos_offset is not None else None
+    in_s = state[0].data_ptr() if state is not None else None
+    in_a = state[1].data_ptr() if state is not None else None
+    if out is None:
+        pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+        start = torch.empty(b, dtype=torch.int32, device=dev)
+        amount = torch.empty(b, dtype=torch.int32, device=dev)
+    else:
+        pos, start, amount = out
+        for t, name in ((pos, "pos"), (start, "start"), (amount, "amount")):
+            _want(t, name, torch.int32, dev)
+        if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
+            raise ValueError("output shapes must be [3, N], [B], [B]")
+    st_ptr = None
+    if device_status is not None:
+        _want(device_status, "device_status", torch.int32, dev)
+        st_ptr = device_status.data_ptr()
+    with torch.cuda.device(dev):
+        _check(lib().cmr_positions_chunk(ids.data_ptr() if n else None, cu_seqlens.data_ptr(), b,
+                                         n, int(image_token_id), RULES[rule], off_ptr, in_s, in_a,
+                                         pos.data_ptr() if n else None,
+                                         start.data_ptr() if b else None,
+                                         amount.data_ptr() if b else None, st_ptr,
+                                         _stream_ptr(dev, stream)), "cmr_positions_chunk")
+    return pos, start, amount
+
+
 def positions_step(cache_len: torch.Tensor, start: torch.Tensor, amount: torch.Tensor,
                    out: Optional[torch.Tensor] = None,
                    stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
@@ -149,17 +214,7 @@ def positions_step(cache_len: torch.Tensor, start: torch.Tensor, amount: torch.T
     return pos
 
 
-def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor,
-              theta: float = 1e7, sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
-              stream: Optional[torch.cuda.Stream] = None):
-    """cmr_rotate_qk, in place.  q: bf16 [L, N, hq, D] (or [N, hq, D]); k likewise
-    with hk heads; pos: int32 [3, N].  Returns (q, k)."""
-    _want(pos, "pos", torch.int32)
-    dev = pos.device
-    if pos.dim() != 2 or pos.shape[0] != 3:
-        raise ValueError("pos must be [3, N]")
-    n = pos.shape[1]
-
+def _qk_shapes(q, k, dev, n):
     def shape_of(t, name):
         if t is None:
             return None
@@ -178,8 +233,59 @@ def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.T
     for s, name in ((qs, "q"), (ks, "k")):
         if s is not None and (s[0] != L or s[1] != n or s[3] != D):
             raise ValueError(f"{name} shape {s} does not match L={L}, N={n}, D={D}")
-    hq = qs[2] if qs else 0
-    hk = ks[2] if ks else 0
+    return L, (qs[2] if qs else 0), (ks[2] if ks else 0), D
+
+
+def rotate_qk_shift(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                    start: torch.Tensor, amount: torch.Tensor,
+                    cu_seqlens: Optional[torch.Tensor] = None,
+                    pos_offset: Optional[torch.Tensor] = None, theta: float = 1e7,
+                    sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """cmr_rotate_qk_shift, in place: the planes of token t of prompt b are the
+    canvas rows at pos_offset[b] + t - cu[b] under (start[b], amount[b]);
+    cu_seqlens=None means one token per sequence (a decode step)."""
+    _want(start, "start", torch.int32)
+    dev = start.device
+    _want(amount, "amount", torch.int32, dev)
+    b = start.numel()
+    if amount.numel() != b:
+        raise ValueError("start and amount must have the same length")
+    ref = q if q is not None else k
+    n = ref.shape[-3] if ref is not None else 0
+    L, hq, hk, D = _qk_shapes(q, k, dev, n)
+    cu_ptr = off_ptr = None
+    if cu_seqlens is not None:
+        _want(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if cu_seqlens.numel() != b + 1:
+            raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+        cu_ptr = cu_seqlens.data_ptr()
+    if pos_offset is not None:
+        _want(pos_offset, "pos_offset", torch.int32, dev)
+        if pos_offset.numel() != b:
+            raise ValueError("pos_offset needs num_seqs entries")
+        off_ptr = pos_offset.data_ptr()
+    sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
+    with torch.cuda.device(dev):
+        _check(lib().cmr_rotate_qk_shift(
+            q.data_ptr() if q is not None and q.numel() else None,
+            k.data_ptr() if k is not None and k.numel() else None, cu_ptr, b, off_ptr,
+            start.data_ptr() if b else None, amount.data_ptr() if b else None, n, L, hq, hk, D,
+            float(theta), sec, int(rot_dim), _stream_ptr(dev, stream)), "cmr_rotate_qk_shift")
+    return q, k
+
+
+def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor,
+              theta: float = 1e7, sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
+              stream: Optional[torch.cuda.Stream] = None):
+    """cmr_rotate_qk, in place.  q: bf16 [L, N, hq, D] (or [N, hq, D]); k likewise
+    with hk heads; pos: int32 [3, N].  Returns (q, k)."""
+    _want(pos, "pos", torch.int32)
+    dev = pos.device
+    if pos.dim() != 2 or pos.shape[0] != 3:
+        raise ValueError("pos must be [3, N]")
+    n = pos.shape[1]
+    L, hq, hk, D = _qk_shapes(q, k, dev, n)
     sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
     with torch.cuda.device(dev):
         _check(lib().cmr_rotate_qk(q.data_ptr() if q is not None and q.numel() else None,

@@ -49,6 +49,68 @@ cmr_status check_device_ptr(const void* p, const char* name) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool ranges_overlap(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+// Checks shared by both rotate entry points; fills the frequency table and the
+// shape fields of `a`.  Returns CMR_OK with a.n_tokens == 0 when there is
+// nothing to do.
+cmr_status check_rotate(void* q, void* k, int64_t n_tokens, int32_t num_layers, int32_t hq,
+                        int32_t hk, int32_t head_dim, double theta, const int32_t sections[3],
+                        int32_t rot_dim, cmr::RotateArgs* a, cmr::FreqTable* table) {
+  if (n_tokens < 0 || num_layers < 0) return fail(CMR_EINVAL, "negative n_tokens or num_layers");
+  if (hq < 0 || hk < 0 || hq + hk < 1) return fail(CMR_EINVAL, "need hq, hk >= 0, hq + hk >= 1");
+  if (head_dim <= 0 || head_dim % 8 != 0) return fail(CMR_EINVAL, "head_dim must be a positive multiple of 8");
+  if (rot_dim < 16 || rot_dim % 16 != 0 || rot_dim > head_dim || rot_dim > 2 * cmr::kMaxFreqs)
+    return fail(CMR_EINVAL, "rot_dim must be a multiple of 16 in [16, min(head_dim, 256)]");
+  if (!(theta > 0.0) || !std::isfinite(theta)) return fail(CMR_EINVAL, "theta must be finite and > 0");
+  if (!sections) return fail(CMR_EINVAL, "sections is required");
+
+  // Frequency -> plane: H takes j = 1, 4, 7, ... (sections[1] of them), W takes
+  // j = 2, 5, 8, ... (sections[2]), T keeps the rest and must count sections[0].
+  const int F = rot_dim / 2;
+  for (int j = 0; j < cmr::kMaxFreqs; ++j) {
+    table->plane[j] = 0;
+    table->inv_freq[j] = 0.0;
+  }
+  if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
+      static_cast<int64_t>(sections[0]) + sections[1] + sections[2] != F)
+    return fail(CMR_EINVAL, "sections must be >= 0 and sum to rot_dim / 2");
+  for (int plane = 1; plane <= 2; ++plane)
+    for (int m = 0; m < sections[plane]; ++m) {
+      const int j = 3 * m + plane;
+      if (j >= F) return fail(CMR_EINVAL, "sections[%d] = %d does not fit the interleave", plane, sections[plane]);
+      table->plane[j] = plane;
+    }
+  for (int j = 0; j < F; ++j) table->inv_freq[j] = std::pow(theta, -2.0 * j / rot_dim);
+
+  const int64_t rows = (static_cast<int64_t>(hq) + hk) * num_layers;  // head rows per token
+  if (rows > INT32_MAX)
+    return fail(CMR_EUNSUPPORTED, "(hq + hk) * num_layers = %lld exceeds INT32_MAX",
+                static_cast<long long>(rows));
+  *a = cmr::RotateArgs{};
+  a->n_tokens = (num_layers == 0) ? 0 : n_tokens;
+  if (a->n_tokens == 0) return CMR_OK;
+  if (hq > 0 && !q) return fail(CMR_EINVAL, "q is required when hq > 0");
+  if (hk > 0 && !k) return fail(CMR_EINVAL, "k is required when hk > 0");
+  if ((hq > 0 && !aligned16(q)) || (hk > 0 && !aligned16(k)))
+    return fail(CMR_EINVAL, "q and k must be 16-byte aligned");
+  cmr_status s;
+  if (hq > 0 && (s = check_device_ptr(q, "q")) != CMR_OK) return s;
+  if (hk > 0 && (s = check_device_ptr(k, "k")) != CMR_OK) return s;
+  a->q = static_cast<uint16_t*>(q);
+  a->k = static_cast<uint16_t*>(k);
+  a->num_layers = num_layers;
+  a->hq = hq;
+  a->hk = hk;
+  a->head_dim = head_dim;
+  a->rot_dim = rot_dim;
+  a->units_per_head = rot_dim / 16;
+  return CMR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -65,7 +127,7 @@ const char* cmr_status_string(cmr_status s) {
 
 const char* cmr_last_error_message(void) { return g_message; }
 
-int32_t cmr_version(void) { return 10000; }  // 1.0.0
+int32_t cmr_version(void) { return 10100; }  // 1.1.0
 
 cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
@@ -90,9 +152,53 @@ cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t 
   }
   if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
   cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
-                                        out_pos, out_start, out_amount, device_status,
+                                        CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
+                                        out_start, out_amount, device_status,
                                         reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "positions launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                               int64_t n_tokens, int32_t image_token_id, int32_t rule,
+                               const int32_t* pos_offset, const int32_t* in_start,
+                               const int32_t* in_amount, int32_t* out_pos, int32_t* out_start,
+                               int32_t* out_amount, int32_t* device_status, cmr_stream_t stream) {
+  if (rule != CMR_RULE_CANVAS && rule != CMR_RULE_QWEN_VL && rule != CMR_RULE_PLANES_1D)
+    return fail(CMR_EINVAL, "unknown rule %d", rule);
+  if (num_seqs < 0 || n_tokens < 0) return fail(CMR_EINVAL, "negative num_seqs or n_tokens");
+  if (n_tokens > INT32_MAX) return fail(CMR_EINVAL, "n_tokens exceeds int32 indexing");
+  if (num_seqs == 0) {
+    if (n_tokens != 0) return fail(CMR_EINVAL, "num_seqs == 0 with n_tokens > 0");
+    return CMR_OK;
+  }
+  if (!cu_seqlens || !out_start || !out_amount)
+    return fail(CMR_EINVAL, "cu_seqlens, out_start and out_amount are required");
+  if (n_tokens > 0 && (!ids || !out_pos)) return fail(CMR_EINVAL, "ids and out_pos are required");
+  // Every CTA of a chunk reads the incoming state while slice 0 writes the
+  // outgoing one, so the two must not share memory.
+  const size_t bytes = static_cast<size_t>(num_seqs) * sizeof(int32_t);
+  for (const int32_t* in : {in_start, in_amount})
+    for (const int32_t* out : {out_start, out_amount})
+      if (in && ranges_overlap(in, out, bytes))
+        return fail(CMR_EINVAL, "incoming and outgoing state must not overlap");
+  cmr_status s;
+  if ((s = check_device_ptr(cu_seqlens, "cu_seqlens")) != CMR_OK) return s;
+  if ((s = check_device_ptr(out_start, "out_start")) != CMR_OK) return s;
+  if ((s = check_device_ptr(out_amount, "out_amount")) != CMR_OK) return s;
+  if (n_tokens > 0) {
+    if ((s = check_device_ptr(ids, "ids")) != CMR_OK) return s;
+    if ((s = check_device_ptr(out_pos, "out_pos")) != CMR_OK) return s;
+  }
+  if (pos_offset && (s = check_device_ptr(pos_offset, "pos_offset")) != CMR_OK) return s;
+  if (in_start && (s = check_device_ptr(in_start, "in_start")) != CMR_OK) return s;
+  if (in_amount && (s = check_device_ptr(in_amount, "in_amount")) != CMR_OK) return s;
+  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule,
+                                        pos_offset, in_start, in_amount, out_pos, out_start,
+                                        out_amount, device_status,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions_chunk launch");
   return CMR_OK;
 }
 
@@ -118,61 +224,44 @@ cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
                          int32_t num_layers, int32_t hq, int32_t hk, int32_t head_dim,
                          double theta, const int32_t sections[3], int32_t rot_dim,
                          cmr_stream_t stream) {
-  if (n_tokens < 0 || num_layers < 0) return fail(CMR_EINVAL, "negative n_tokens or num_layers");
-  if (hq < 0 || hk < 0 || hq + hk < 1) return fail(CMR_EINVAL, "need hq, hk >= 0, hq + hk >= 1");
-  if (head_dim <= 0 || head_dim % 8 != 0) return fail(CMR_EINVAL, "head_dim must be a positive multiple of 8");
-  if (rot_dim < 16 || rot_dim % 16 != 0 || rot_dim > head_dim || rot_dim > 2 * cmr::kMaxFreqs)
-    return fail(CMR_EINVAL, "rot_dim must be a multiple of 16 in [16, min(head_dim, 256)]");
-  if (!(theta > 0.0) || !std::isfinite(theta)) return fail(CMR_EINVAL, "theta must be finite and > 0");
-  if (!sections) return fail(CMR_EINVAL, "sections is required");
-
-  // Frequency -> plane: H takes j = 1, 4, 7, ... (sections[1] of them), W takes
-  // j = 2, 5, 8, ... (sections[2]), T keeps the rest and must count sections[0].
-  const int F = rot_dim / 2;
+  cmr::RotateArgs a;
   cmr::FreqTable table;
-  for (int j = 0; j < cmr::kMaxFreqs; ++j) {
-    table.plane[j] = 0;
-    table.inv_freq[j] = 0.0;
-  }
-  if (sections[0] < 0 || sections[1] < 0 || sections[2] < 0 ||
-      static_cast<int64_t>(sections[0]) + sections[1] + sections[2] != F)
-    return fail(CMR_EINVAL, "sections must be >= 0 and sum to rot_dim / 2");
-  for (int plane = 1; plane <= 2; ++plane)
-    for (int m = 0; m < sections[plane]; ++m) {
-      const int j = 3 * m + plane;
-      if (j >= F) return fail(CMR_EINVAL, "sections[%d] = %d does not fit the interleave", plane, sections[plane]);
-      table.plane[j] = plane;
-    }
-  for (int j = 0; j < F; ++j) table.inv_freq[j] = std::pow(theta, -2.0 * j / rot_dim);
-
-  const int64_t rows = (static_cast<int64_t>(hq) + hk) * num_layers;  // head rows per token
-  if (rows > INT32_MAX)
-    return fail(CMR_EUNSUPPORTED, "(hq + hk) * num_layers = %lld exceeds INT32_MAX",
-                static_cast<long long>(rows));
-  if (n_tokens == 0 || num_layers == 0) return CMR_OK;
+  cmr_status s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections,
+                              rot_dim, &a, &table);
+  if (s != CMR_OK || a.n_tokens == 0) return s;
   if (!pos) return fail(CMR_EINVAL, "pos is required");
-  if (hq > 0 && !q) return fail(CMR_EINVAL, "q is required when hq > 0");
-  if (hk > 0 && !k) return fail(CMR_EINVAL, "k is required when hk > 0");
-  if ((hq > 0 && !aligned16(q)) || (hk > 0 && !aligned16(k)))
-    return fail(CMR_EINVAL, "q and k must be 16-byte aligned");
-  cmr_status s;
   if ((s = check_device_ptr(pos, "pos")) != CMR_OK) return s;
-  if (hq > 0 && (s = check_device_ptr(q, "q")) != CMR_OK) return s;
-  if (hk > 0 && (s = check_device_ptr(k, "k")) != CMR_OK) return s;
-
-  cmr::RotateArgs a{};
-  a.q = static_cast<uint16_t*>(q);
-  a.k = static_cast<uint16_t*>(k);
   a.pos = pos;
-  a.n_tokens = n_tokens;
-  a.num_layers = num_layers;
-  a.hq = hq;
-  a.hk = hk;
-  a.head_dim = head_dim;
-  a.rot_dim = rot_dim;
-  a.units_per_head = rot_dim / 16;
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens, int32_t num_seqs,
+                               const int32_t* pos_offset, const int32_t* start,
+                               const int32_t* amount, int64_t n_tokens, int32_t num_layers,
+                               int32_t hq, int32_t hk, int32_t head_dim, double theta,
+                               const int32_t sections[3], int32_t rot_dim, cmr_stream_t stream) {
+  cmr::RotateArgs a;
+  cmr::FreqTable table;
+  cmr_status s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections,
+                              rot_dim, &a, &table);
+  if (s != CMR_OK || a.n_tokens == 0) return s;
+  if (num_seqs <= 0) return fail(CMR_EINVAL, "num_seqs must be > 0 when there are tokens");
+  if (!cu_seqlens && num_seqs != n_tokens)
+    return fail(CMR_EINVAL, "without cu_seqlens every sequence holds one token (num_seqs == n_tokens)");
+  if (!start || !amount) return fail(CMR_EINVAL, "start and amount are required");
+  if (cu_seqlens && (s = check_device_ptr(cu_seqlens, "cu_seqlens")) != CMR_OK) return s;
+  if (pos_offset && (s = check_device_ptr(pos_offset, "pos_offset")) != CMR_OK) return s;
+  if ((s = check_device_ptr(start, "start")) != CMR_OK) return s;
+  if ((s = check_device_ptr(amount, "amount")) != CMR_OK) return s;
+  a.cu = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.pos_offset = pos_offset;
+  a.start = start;
+  a.amount = amount;
+  cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_qk_shift launch");
   return CMR_OK;
 }
 

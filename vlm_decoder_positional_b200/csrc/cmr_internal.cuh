@@ -30,17 +30,27 @@ struct FreqTable {
 struct RotateArgs {
   uint16_t* q;  // bf16 bits [L, N, hq, D]
   uint16_t* k;  // bf16 bits [L, N, hk, D]
-  const int32_t* pos;  // [3, N]
+  const int32_t* pos;  // [3, N], or nullptr when the planes come from the shift state
+  // shift state (planes derived in the kernel): token t of prompt b sits at
+  // absolute index pos_offset[b] + t - cu[b]; cu == nullptr: one token each
+  const int32_t* cu;
+  const int32_t* pos_offset;
+  const int32_t* start;
+  const int32_t* amount;
+  int32_t num_seqs;
   int64_t n_tokens;
   int32_t num_layers;
   int32_t hq, hk, head_dim, rot_dim;
   int32_t units_per_head;  // rot_dim / 16: threads per token, 8 frequencies each
+  int32_t head_groups;      // work items per token (set at launch)
+  int32_t heads_per_group;
 };
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
-                             int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
-                             int32_t* out_start, int32_t* out_amount, int32_t* device_status,
-                             cudaStream_t stream);
+                             int64_t n_tokens, int32_t image_token_id, int32_t rule,
+                             const int32_t* pos_offset, const int32_t* in_start,
+                             const int32_t* in_amount, int32_t* out_pos, int32_t* out_start,
+                             int32_t* out_amount, int32_t* device_status, cudaStream_t stream);
 
 cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start,
                                   const int32_t* amount, int32_t num_seqs, int32_t* out_pos,

@@ -3,19 +3,22 @@
 // Rule: the canvas table of the HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI,
 // section "How the VLM rides the text-only engine", with start = O + 67 and
 // amount = start - (O + 9) from the Core AI port notes ("The canvas rule and
-// why the gate is on the planes").
+// why the gate is on the planes").  The port notes' CoreAIKit section gives
+// Qwen-VL's shift for comparison (+64 from the pads, 56: start = O + 65), and
+// the LiteRT card's runtime uses plain 1-D positions; both are selectable.
 //
-// Work split: CTA (b, s) owns slice s of prompt b.  To know the origin O it
-// scans the prompt's ids from index 0 up to the end of its own slice (slice 0
-// scans the whole prompt, since it also writes start/amount), in chunks of
-// 8192 ids (16 loads in flight per thread), and stops at the first chunk that
-// holds a marker.  A marker past
-// the slice cannot change the slice's planes (every token there is p < O ->
-// (p, p, p), the same as text-only), so no CTA waits on another and there is
-// no scratch memory and no atomics.  Ids re-read by later slices hit L2.
+// Work split: CTA (b, s) owns slice s of prompt chunk b.  When the chunk's
+// sequence has no frame yet, the CTA finds the origin by scanning the chunk's
+// ids from index 0 up to the end of its own slice (slice 0 scans the whole
+// chunk, since it also writes the state), in chunks of 8192 ids (16 loads in
+// flight per thread), and stops at the first chunk that holds a marker.  A
+// marker past the slice cannot change the slice's planes (every token there
+// is p < O -> (p, p, p), the same as text-only), so no CTA waits on another
+// and there is no scratch memory and no atomics on data.  Ids re-read by later
+// slices hit L2.
 #include <climits>
 
-#include "cmr_internal.cuh"
+#include "canvas.cuh"
 
 namespace cmr {
 namespace {
@@ -25,33 +28,7 @@ constexpr int kIdsPerThread = 16;
 constexpr int kScanChunk = kPosThreads * kIdsPerThread;  // 8192 ids per step
 constexpr int kSliceTarget = 2048;                       // tokens per CTA (target)
 constexpr int kMaxSlices = 65535;                        // gridDim.y limit
-
-struct Planes {
-  int32_t t, h, w;
-};
-
-// Row of the canvas table for local index p.  The "after the frame" row is
-// tested first so that any (start, amount) pair gives one answer.
-__device__ __forceinline__ Planes canvas_row(int64_t p, int64_t origin, int64_t start,
-                                             int64_t amount) {
-  if (p >= start) {
-    const int32_t v = static_cast<int32_t>(p - amount);
-    return {v, v, v};
-  }
-  const int64_t d = p - origin;  // offset into the frame
-  const int32_t o = static_cast<int32_t>(origin);
-  if (d < 0) {
-    const int32_t v = static_cast<int32_t>(p);
-    return {v, v, v};
-  }
-  if (d == 0) return {o, o - 1, o - 1};  // <image>
-  if (d <= kGridRows) {                  // image row k = d - 1
-    const int32_t k = static_cast<int32_t>(d - 1);
-    return {o, o + k / kGridSide, o + k % kGridSide};
-  }
-  if (d == kGridRows + 1) return {o, o + kGridSide, o + kGridSide};  // </image>
-  return {o, o, o};  // the "\n" after </image>
-}
+constexpr int kQwenVlFrameShift = kGridRows + 1;         // start = O + 65
 
 // Smallest local index in [0, scan_end) whose id is the marker, or -1.
 // Block-uniform result; all threads of the CTA must call it.
@@ -84,9 +61,12 @@ __device__ __forceinline__ int64_t find_origin(const int32_t* __restrict__ seq, 
 
 __global__ void __launch_bounds__(kPosThreads)
     canvas_positions_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
-                            int32_t num_seqs, int64_t n_tokens, int32_t marker,
-                            int32_t* __restrict__ pos, int32_t* __restrict__ out_start,
-                            int32_t* __restrict__ out_amount, int32_t* __restrict__ status) {
+                            int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t rule,
+                            const int32_t* __restrict__ pos_offset,
+                            const int32_t* __restrict__ in_start,
+                            const int32_t* __restrict__ in_amount, int32_t* __restrict__ pos,
+                            int32_t* __restrict__ out_start, int32_t* __restrict__ out_amount,
+                            int32_t* __restrict__ status) {
   __shared__ int s_warp_min[kPosThreads / 32];
   const int32_t b = blockIdx.x;
   const int64_t first = __ldg(cu + b);
@@ -103,16 +83,24 @@ __global__ void __launch_bounds__(kPosThreads)
   const int64_t p1 = min(len, p0 + per);
   if (blockIdx.y != 0 && p0 >= p1) return;
 
-  const int64_t scan_end = (blockIdx.y == 0) ? len : p1;
-  const int64_t origin = find_origin(ids + first, scan_end, marker, s_warp_min);
-
-  int64_t start, amount;
-  if (origin >= 0) {
-    start = origin + kFrameTokens;
-    amount = start - (origin + kCanvasSpan);
-  } else {
+  // The sequence's state before this chunk: (2^30, 0) while no frame is known.
+  const int64_t offset = pos_offset ? __ldg(pos_offset + b) : 0;
+  int64_t start = in_start ? __ldg(in_start + b) : kTextOnlyStart;
+  int64_t amount = in_amount ? __ldg(in_amount + b) : 0;
+  if (rule == CMR_RULE_PLANES_1D) {
     start = kTextOnlyStart;
     amount = 0;
+  } else if (start >= kTextOnlyStart) {
+    const int64_t scan_end = (blockIdx.y == 0) ? len : p1;
+    const int64_t m = find_origin(ids + first, scan_end, marker, s_warp_min);
+    if (m >= 0) {
+      const int64_t origin = offset + m;
+      start = origin + (rule == CMR_RULE_QWEN_VL ? kQwenVlFrameShift : kFrameTokens);
+      amount = start - (origin + kCanvasSpan);
+    } else {
+      start = kTextOnlyStart;
+      amount = 0;
+    }
   }
   if (blockIdx.y == 0 && threadIdx.x == 0) {
     out_start[b] = static_cast<int32_t>(start);
@@ -122,16 +110,16 @@ __global__ void __launch_bounds__(kPosThreads)
   int32_t* __restrict__ pt = pos + first;
   int32_t* __restrict__ ph = pos + n_tokens + first;
   int32_t* __restrict__ pw = pos + 2 * n_tokens + first;
-  if (origin < 0) {
+  if (start >= kTextOnlyStart) {
     for (int64_t p = p0 + threadIdx.x; p < p1; p += kPosThreads) {
-      const int32_t v = static_cast<int32_t>(p);
+      const int32_t v = static_cast<int32_t>(offset + p);
       pt[p] = v;
       ph[p] = v;
       pw[p] = v;
     }
   } else {
     for (int64_t p = p0 + threadIdx.x; p < p1; p += kPosThreads) {
-      const Planes r = canvas_row(p, origin, start, amount);
+      const Planes r = canvas_row(offset + p, start, amount);
       pt[p] = r.t;
       ph[p] = r.h;
       pw[p] = r.w;
@@ -145,11 +133,9 @@ __global__ void canvas_positions_step_kernel(const int32_t* __restrict__ cache_l
                                              int32_t num_seqs, int32_t* __restrict__ pos) {
   for (int64_t b = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; b < num_seqs;
        b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t s = __ldg(start + b);
-    const int64_t a = __ldg(amount + b);
-    // The engine binds only start and amount; the origin follows from
-    // amount = start - (O + 9).
-    const Planes r = canvas_row(__ldg(cache_len + b), s - a - kCanvasSpan, s, a);
+    // The engine binds only start and amount; canvas_row recovers the origin
+    // from amount = start - (O + 9).
+    const Planes r = canvas_row(__ldg(cache_len + b), __ldg(start + b), __ldg(amount + b));
     pos[b] = r.t;
     pos[num_seqs + b] = r.h;
     pos[2 * static_cast<int64_t>(num_seqs) + b] = r.w;
@@ -159,17 +145,18 @@ __global__ void canvas_positions_step_kernel(const int32_t* __restrict__ cache_l
 }  // namespace
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
-                             int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
-                             int32_t* out_start, int32_t* out_amount, int32_t* device_status,
-                             cudaStream_t stream) {
+                             int64_t n_tokens, int32_t image_token_id, int32_t rule,
+                             const int32_t* pos_offset, const int32_t* in_start,
+                             const int32_t* in_amount, int32_t* out_pos, int32_t* out_start,
+                             int32_t* out_amount, int32_t* device_status, cudaStream_t stream) {
   if (num_seqs == 0) return cudaSuccess;
   const int64_t avg = (n_tokens + num_seqs - 1) / num_seqs;
   int64_t slices = (avg + kSliceTarget - 1) / kSliceTarget;
   slices = slices < 1 ? 1 : (slices > kMaxSlices ? kMaxSlices : slices);
   dim3 grid(static_cast<unsigned>(num_seqs), static_cast<unsigned>(slices));
-  canvas_positions_kernel<<<grid, kPosThreads, 0, stream>>>(ids, cu_seqlens, num_seqs, n_tokens,
-                                                            image_token_id, out_pos, out_start,
-                                                            out_amount, device_status);
+  canvas_positions_kernel<<<grid, kPosThreads, 0, stream>>>(
+      ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule, pos_offset, in_start, in_amount,
+      out_pos, out_start, out_amount, device_status);
   return cudaGetLastError();
 }
 

@@ -1,4 +1,6 @@
 // Fused cos/sin + rotate-half M-RoPE of Q and K, in place, on sm_100a.
+// The planes come from pos [3, N] (cmr_rotate_qk) or are derived in the kernel
+// from each prompt's (start, amount) state (cmr_rotate_qk_shift).
 //
 // Math (HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "What it is": planes
 // T, H, W with interleaved sections [11, 11, 10]; port notes: the decoder's
@@ -21,12 +23,14 @@
 // is 8 tokens x 64 contiguous bytes (whole 32-B sectors), and the x / partner
 // loads of one head row together cover its 128-B line.  kBatch head rows are
 // loaded (two 16-byte loads each, evict-first) before any is rotated and
-// stored back (two 16-byte stores each).
+// stored back (two 16-byte stores each).  When a batch has too few tokens to
+// fill the GPU (decode), each token's heads are split into groups handled by
+// different threads, each computing the same 8 cos/sin for its group.
 #include <cuda_bf16.h>
 
 #include <mutex>
 
-#include "cmr_internal.cuh"
+#include "canvas.cuh"
 
 namespace cmr {
 namespace {
@@ -76,6 +80,39 @@ __device__ __forceinline__ void rotate_unit(uint4& x1, uint4& x2, const float (&
   }
 }
 
+// Planes (T, H, W) of token t: read from pos [3, N], or derived from the
+// shift state of the token's prompt (binary search of t in cu_seqlens).
+template <bool kFromShift>
+__device__ __forceinline__ void token_planes(const RotateArgs& a, int64_t t, int32_t& p0,
+                                             int32_t& p1, int32_t& p2) {
+  if constexpr (!kFromShift) {
+    p0 = __ldg(a.pos + t);
+    p1 = __ldg(a.pos + a.n_tokens + t);
+    p2 = __ldg(a.pos + 2 * a.n_tokens + t);
+  } else {
+    int32_t b = static_cast<int32_t>(t);
+    int64_t local = 0;
+    if (a.cu != nullptr) {  // last b with cu[b] <= t; cu[0] = 0 <= t < cu[num_seqs]
+      int32_t lo = 0, hi = a.num_seqs;
+      while (hi - lo > 1) {
+        const int32_t mid = (lo + hi) >> 1;
+        if (__ldg(a.cu + mid) <= t)
+          lo = mid;
+        else
+          hi = mid;
+      }
+      b = lo;
+      local = t - __ldg(a.cu + b);
+    }
+    const int64_t p = (a.pos_offset ? __ldg(a.pos_offset + b) : 0) + local;
+    const Planes r = canvas_row(p, __ldg(a.start + b), __ldg(a.amount + b));
+    p0 = r.t;
+    p1 = r.h;
+    p2 = r.w;
+  }
+}
+
+template <bool kFromShift>
 __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
     rotate_qk_kernel(const RotateArgs args, const FreqTable table) {
   __shared__ double s_inv[kMaxFreqs];
@@ -88,14 +125,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
   __syncthreads();  // the only barrier: the tables are read-only from here on
 
   const int U = args.units_per_head;
-  const int tokens_per_cta = kThreads / U;
+  const int items_per_cta = kThreads / U;
   const int local = threadIdx.x / U;
   const int u = threadIdx.x - local * U;
-  if (local >= tokens_per_cta) return;  // spare threads when U does not divide kThreads
+  if (local >= items_per_cta) return;  // spare threads when U does not divide kThreads
 
   const int64_t N = args.n_tokens;
   const int H = args.hq + args.hk;
-  const int J = H * args.num_layers;  // head rows per token
+  const int G = args.head_groups;
+  const int hpg = args.heads_per_group;
   const int64_t D = args.head_dim;
   const int64_t q_tok = static_cast<int64_t>(args.hq) * D;  // elements per token
   const int64_t k_tok = static_cast<int64_t>(args.hk) * D;
@@ -103,24 +141,28 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
   const int64_t k_layer = N * k_tok;
   const int half4 = F / 8;  // partner offset in 16-byte vectors
 
-  const int64_t t_step = static_cast<int64_t>(gridDim.x) * tokens_per_cta;
-  int64_t t = static_cast<int64_t>(blockIdx.x) * tokens_per_cta + local;
-  // Planes of the current token, loaded one token ahead so that their latency
-  // overlaps the previous token's head rows.
+  // Work item v = g * N + t: the head rows of head group g of token t, in
+  // every layer.  With one group (large batches) an item is a whole token.
+  const int64_t n_items = N * G;
+  const int64_t v_step = static_cast<int64_t>(gridDim.x) * items_per_cta;
+  int64_t v = static_cast<int64_t>(blockIdx.x) * items_per_cta + local;
+  // Planes of the current item's token, loaded one item ahead so that their
+  // latency overlaps the previous item's head rows.
   int32_t p0 = 0, p1 = 0, p2 = 0;
-  if (t < N) {
-    p0 = __ldg(args.pos + t);
-    p1 = __ldg(args.pos + N + t);
-    p2 = __ldg(args.pos + 2 * N + t);
-  }
-  for (; t < N; t += t_step) {
+  if (v < n_items) token_planes<kFromShift>(args, G == 1 ? v : v % N, p0, p1, p2);
+  for (; v < n_items; v += v_step) {
+    const int64_t g = (G == 1) ? 0 : v / N;
+    const int64_t t = v - g * N;
+    const int h_lo = static_cast<int>(g) * hpg;
+    const int h_hi = min(H, h_lo + hpg);
+    const int J = (h_hi - h_lo) * args.num_layers;  // head rows of this item
     // Base of this thread's unit in head 0 of layer 0; K rows are indexed by
     // h - hq, folded into the base so that row h sits at base + h * D.
     uint16_t* const q_base = args.q + t * q_tok + 8 * u;
     uint16_t* const k_base = args.k + t * k_tok + 8 * u - static_cast<int64_t>(args.hq) * D;
 
     // First batch of head rows in flight before the cos/sin work below.
-    int h = 0, l = 0;  // head row of the next job: head h of layer l
+    int h = h_lo, l = 0;  // head row of the next job: head h of layer l
     uint4 x1[kBatch], x2[kBatch];
     uint4* ptr[kBatch];
     auto load_batch = [&](int j0) {
@@ -132,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
           ptr[b] = reinterpret_cast<uint4*>(row + h * D);
           x1[b] = __ldcs(ptr[b]);
           x2[b] = __ldcs(ptr[b] + half4);
-          if (++h == H) {
-            h = 0;
+          if (++h == h_hi) {
+            h = h_lo;
             ++l;
           }
         }
@@ -149,12 +191,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
       const int pl = s_plane[j];
       cos_sin(pl == 0 ? p0 : (pl == 1 ? p1 : p2), s_inv[j], c[e], s[e]);
     }
-    const int64_t tn = t + t_step;
-    if (tn < N) {
-      p0 = __ldg(args.pos + tn);
-      p1 = __ldg(args.pos + N + tn);
-      p2 = __ldg(args.pos + 2 * N + tn);
-    }
+    const int64_t vn = v + v_step;
+    if (vn < n_items) token_planes<kFromShift>(args, G == 1 ? vn : vn % N, p0, p1, p2);
 
     for (int j0 = 0;;) {
 #pragma unroll
@@ -175,40 +213,59 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
 struct OccupancyCache {
   std::mutex mu;
   int device = -1;
-  int ctas = 0;
+  int ctas[2] = {0, 0};
 };
 OccupancyCache g_occ[64];
 
-// CTAs resident on the whole device at full occupancy (cached per device).
-cudaError_t resident_ctas(int* total) {
+// CTAs of each variant resident on the whole device at full occupancy
+// (cached per device).
+cudaError_t resident_ctas(bool from_shift, int* total) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   OccupancyCache& c = g_occ[dev & 63];
   std::lock_guard<std::mutex> lock(c.mu);
   if (c.device != dev) {
-    int sms = 0, per_sm = 0;
+    int sms = 0, per_sm[2] = {0, 0};
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rotate_qk_kernel, kThreads, 0);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[0], rotate_qk_kernel<false>,
+                                                      kThreads, 0);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[1], rotate_qk_kernel<true>,
+                                                      kThreads, 0);
     if (e != cudaSuccess) return e;
     c.device = dev;
-    c.ctas = sms * (per_sm > 0 ? per_sm : 1);
+    for (int i = 0; i < 2; ++i) c.ctas[i] = sms * (per_sm[i] > 0 ? per_sm[i] : 1);
   }
-  *total = c.ctas;
+  *total = c.ctas[from_shift ? 1 : 0];
   return cudaSuccess;
 }
 
 }  // namespace
 
-cudaError_t launch_rotate_qk(const RotateArgs& a, const FreqTable& table, cudaStream_t stream) {
+cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream) {
+  RotateArgs a = in;
+  const bool from_shift = a.pos == nullptr;
   int max_ctas = 0;
-  cudaError_t e = resident_ctas(&max_ctas);
+  cudaError_t e = resident_ctas(from_shift, &max_ctas);
   if (e != cudaSuccess) return e;
-  const int64_t tokens_per_cta = kThreads / a.units_per_head;
-  const int64_t needed = (a.n_tokens + tokens_per_cta - 1) / tokens_per_cta;
+  const int64_t items_per_cta = kThreads / a.units_per_head;
+  // Split each token's heads into groups only when there are too few tokens
+  // to fill one wave of resident CTAs.
+  const int heads = a.hq + a.hk;
+  const int64_t wave_items = static_cast<int64_t>(max_ctas) * items_per_cta;
+  int64_t groups = (wave_items + a.n_tokens - 1) / a.n_tokens;
+  groups = groups < 1 ? 1 : (groups > heads ? heads : groups);
+  a.heads_per_group = static_cast<int32_t>((heads + groups - 1) / groups);
+  a.head_groups = (heads + a.heads_per_group - 1) / a.heads_per_group;
+  const int64_t items = a.n_tokens * a.head_groups;
+  const int64_t needed = (items + items_per_cta - 1) / items_per_cta;
   const int64_t ctas = needed < max_ctas ? needed : max_ctas;
-  rotate_qk_kernel<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
+  if (from_shift)
+    rotate_qk_kernel<true><<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
+  else
+    rotate_qk_kernel<false><<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
   return cudaGetLastError();
 }
 
