@@ -290,19 +290,46 @@ def run_ours(args):
     amount = torch.empty(b, dtype=torch.int32, device=dev)
     decode = wl.cache_len is not None
     cache_len = torch.from_numpy(wl.cache_len).to(dev) if decode else None
-    pos_step = torch.empty((3, b), dtype=torch.int32, device=dev) if decode else None
     stream = torch.cuda.current_stream(dev)
     tokens_per_step = wl.qk_tokens
     rot_b = rotate_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim)
 
+    if decode:
+        # The prompts' (start, amount) come from their prefill, once; a decode
+        # step is one launch that derives each new token's planes in the
+        # kernel from (cache_len, start, amount) and rotates it.
+        cmr.positions(ids, cu, wl.image_token_id, out=(pos, start, amount))
+        plan = [("rotate", lambda: cmr.rotate_qk_shift(wl.q, wl.k, start, amount,
+                                                       pos_offset=cache_len, theta=wl.theta,
+                                                       sections=wl.sections,
+                                                       rot_dim=wl.rot_dim))]
+    else:
+        plan = [("positions", lambda: cmr.positions(ids, cu, wl.image_token_id,
+                                                    out=(pos, start, amount))),
+                ("rotate", lambda: cmr.rotate_qk(wl.q, wl.k, pos, wl.theta, wl.sections,
+                                                 wl.rot_dim))]
+    calls = dict(plan)
+    if args.launch == "graph":
+        # one CUDA graph per call, each holding its single kernel launch
+        for fn in calls.values():
+            fn()
+        torch.cuda.synchronize(dev)
+        graphs = {}
+        for name, fn in plan:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs[name] = g
+        calls = {name: g.replay for name, g in graphs.items()}
+
     def step(ev=None):
         if ev is not None:
             ev[2].record(stream)
-        p, s, a = cmr.positions(ids, cu, wl.image_token_id, out=(pos, start, amount))
-        pr = cmr.positions_step(cache_len, s, a, out=pos_step) if decode else p
+        if "positions" in calls:
+            calls["positions"]()
         if ev is not None:
             ev[0].record(stream)
-        cmr.rotate_qk(wl.q, wl.k, pr, wl.theta, wl.sections, wl.rot_dim)
+        calls["rotate"]()
         if ev is not None:
             ev[1].record(stream)
 
@@ -331,7 +358,7 @@ def run_ours(args):
     ms_max = shard.max_over_ranks(ms, dist, dev)
     # tokens processed by all ranks in one step
     tokens_all = tokens_per_step * world if args.scaling == "weak" else global_tokens
-    launches = args.steps * (3 if decode else 2)
+    launches = args.steps * len(plan)
 
     # end to end through the public API from pinned host memory
     e2e = run_e2e(args, wl, dev, stream, dist, tokens_all)
@@ -353,6 +380,7 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1) bf16 Q/K, uniform text ids, one 448x448 frame "
                     "per prompt)",
             "config": {"workload": workload_label(wl), "global_batch": tokens_all,
+                       "launch": args.launch,
                        "seq_len": n // max(b, 1),
                        "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'whole prompts split over ranks'}, no data-path collective)",
                        "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
@@ -389,26 +417,37 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
     h_q.copy_(wl.q)
     h_k.copy_(wl.k)
     decode = wl.cache_len is not None
-    h_cl = torch.from_numpy(wl.cache_len).pin_memory() if decode else None
     npos = wl.qk_tokens
     h_pos = torch.empty((3, npos), dtype=torch.int32, pin_memory=True)
     h_start = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
     h_amount = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
+    if decode:
+        # per decode step the host sends the new tokens' Q/K and each
+        # sequence's length and (start, amount) state, known from its prefill
+        _, s, a = cmr.positions(h_ids.to(dev), h_cu.to(dev), wl.image_token_id)
+        h_start.copy_(s)
+        h_amount.copy_(a)
+        h_cl = torch.from_numpy(wl.cache_len).pin_memory()
 
     def step():
-        ids = h_ids.to(dev, non_blocking=True)
-        cu = h_cu.to(dev, non_blocking=True)
         q = h_q.to(dev, non_blocking=True)
         k = h_k.to(dev, non_blocking=True)
-        pos, start, amount = cmr.positions(ids, cu, wl.image_token_id)
         if decode:
-            pos = cmr.positions_step(h_cl.to(dev, non_blocking=True), start, amount)
-        cmr.rotate_qk(q, k, pos, wl.theta, wl.sections, wl.rot_dim)
+            cl = h_cl.to(dev, non_blocking=True)
+            start = h_start.to(dev, non_blocking=True)
+            amount = h_amount.to(dev, non_blocking=True)
+            cmr.rotate_qk_shift(q, k, start, amount, pos_offset=cl, theta=wl.theta,
+                                sections=wl.sections, rot_dim=wl.rot_dim)
+        else:
+            ids = h_ids.to(dev, non_blocking=True)
+            cu = h_cu.to(dev, non_blocking=True)
+            pos, start, amount = cmr.positions(ids, cu, wl.image_token_id)
+            cmr.rotate_qk(q, k, pos, wl.theta, wl.sections, wl.rot_dim)
+            h_pos.copy_(pos, non_blocking=True)
+            h_start.copy_(start, non_blocking=True)
+            h_amount.copy_(amount, non_blocking=True)
         h_q.copy_(q, non_blocking=True)
         h_k.copy_(k, non_blocking=True)
-        h_pos.copy_(pos, non_blocking=True)
-        h_start.copy_(start, non_blocking=True)
-        h_amount.copy_(amount, non_blocking=True)
 
     step()
     torch.cuda.synchronize(dev)
@@ -421,13 +460,17 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
     z.record(stream)
     torch.cuda.synchronize(dev)
     ms = shard.max_over_ranks(a.elapsed_time(z), dist, dev)
-    h2d = (h_ids.numel() * 4 + h_cu.numel() * 4 + h_q.numel() * 2 + h_k.numel() * 2
-           + (h_cl.numel() * 4 if decode else 0))
-    d2h = h_q.numel() * 2 + h_k.numel() * 2 + h_pos.numel() * 4 + 8 * wl.num_seqs
+    if decode:
+        h2d = h_q.numel() * 2 + h_k.numel() * 2 + 12 * wl.num_seqs
+        d2h = h_q.numel() * 2 + h_k.numel() * 2
+    else:
+        h2d = h_ids.numel() * 4 + h_cu.numel() * 4 + h_q.numel() * 2 + h_k.numel() * 2
+        d2h = h_q.numel() * 2 + h_k.numel() * 2 + h_pos.numel() * 4 + 8 * wl.num_seqs
     return {"value": tokens_all * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
-            "path": "pinned host -> cmr.positions + cmr.rotate_qk -> pinned host"}
+            "path": ("pinned host -> cmr.rotate_qk_shift -> pinned host" if decode else
+                     "pinned host -> cmr.positions + cmr.rotate_qk -> pinned host")}
 
 
 def main():
@@ -442,6 +485,9 @@ def main():
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: a full batch per GPU (default); strong: one batch split by "
                          "whole prompts")
+    ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
+                    help="graph: replay a captured CUDA graph per call (default); eager: "
+                         "launch through the Python binding every step")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)

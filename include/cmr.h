@@ -52,6 +52,7 @@ typedef enum cmr_status {
 
 /* Bits a kernel ORs into the optional device status word. */
 #define CMR_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens not 0 .. n_tokens, non-decreasing */
+#define CMR_DEVICE_CACHE_RANGE 2    /* a token's cache index or slot outside the cache */
 
 /* Position rules for cmr_positions_chunk. */
 #define CMR_RULE_CANVAS 0    /* this model's canvas rule: start = O + 67, amount 58 */
@@ -207,6 +208,41 @@ CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqle
                                        int32_t hk, int32_t head_dim, double theta,
                                        const int32_t sections[3], int32_t rot_dim,
                                        cmr_stream_t stream);
+
+/* Rotate Q in place and write each token's rotated K row and its V row into
+ * a KV cache, in one pass: the step after the rotation in the full-attention
+ * layers (HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides
+ * the text-only engine": keyCache / valueCache [6, 1, 2, -1, 256], the 6
+ * full-attention layers, context up to 4,096).  Token t of prompt b sits at
+ * absolute index p = pos_offset[b] + t - cu[b]; its planes are the canvas rows
+ * at p under (start[b], amount[b]) as in cmr_rotate_qk_shift; its rows land at
+ *   k_cache[l, slot, h, p, :] = K[l, t, h, :] rotated (all head_dim dims)
+ *   v_cache[l, slot, h, p, :] = V[l, t, h, :]
+ * with slot = cache_slot[b] (or b when cache_slot is NULL).  K and V are not
+ * modified.  A token whose p or slot falls outside the cache writes no K/V row
+ * and ORs CMR_DEVICE_CACHE_RANGE into device_status.
+ *
+ *   q                  device bf16 [num_layers, n_tokens, hq, head_dim], rotated in place
+ *   k, v               device bf16 [num_layers, n_tokens, hk, head_dim], read only
+ *   k_cache, v_cache   device bf16 [num_layers, cache_seqs, hk, cache_ctx, head_dim]
+ *   cache_slot         device int32 [num_seqs], or NULL
+ *   cache_seqs, cache_ctx  > 0
+ *   cu_seqlens, num_seqs, pos_offset, start, amount   as in cmr_rotate_qk_shift
+ *   the rest           as in cmr_rotate_qk
+ * All of q, k, v, k_cache, v_cache 16-byte aligned; the caches must not
+ * overlap q, k or v.
+ * Errors: as cmr_rotate_qk_shift, plus CMR_EINVAL for missing or misaligned
+ * v / caches or non-positive cache sizes. */
+CMR_API cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v,
+                                       const int32_t* cu_seqlens, int32_t num_seqs,
+                                       const int32_t* pos_offset, const int32_t* start,
+                                       const int32_t* amount, int64_t n_tokens,
+                                       int32_t num_layers, int32_t hq, int32_t hk,
+                                       int32_t head_dim, double theta,
+                                       const int32_t sections[3], int32_t rot_dim,
+                                       void* k_cache, void* v_cache, int32_t cache_seqs,
+                                       int32_t cache_ctx, const int32_t* cache_slot,
+                                       int32_t* device_status, cmr_stream_t stream);
 
 /* Static, never-null description of a status code. */
 CMR_API const char* cmr_status_string(cmr_status s);

@@ -189,3 +189,48 @@ def f64_to_bf16(values):
     flat = np.asarray(values, dtype=np.float64).ravel()
     out = np.array([lib.oracle_f64_to_bf16(float(v)) for v in flat], dtype=np.uint16)
     return out.reshape(np.shape(values))
+
+
+def token_index(n_tokens, num_seqs, cu_seqlens=None, pos_offset=None):
+    """Sequence b and absolute index p of every packed token (cu_seqlens None:
+    token b is sequence b)."""
+    if cu_seqlens is None:
+        b = np.arange(n_tokens, dtype=np.int64)
+        local = np.zeros(n_tokens, dtype=np.int64)
+    else:
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+        b = np.repeat(np.arange(num_seqs), np.diff(cu))
+        local = np.arange(n_tokens, dtype=np.int64) - cu[b]
+    off = np.zeros(num_seqs, np.int64) if pos_offset is None else np.asarray(pos_offset, np.int64)
+    return b, off[b] + local
+
+
+def rotate_qk_cache(q_bits, k_bits, v_bits, start, amount, k_cache_bits, v_cache_bits,
+                    cu_seqlens=None, pos_offset=None, cache_slot=None, theta=1e7,
+                    sections=(11, 11, 10), rot_dim=64):
+    """Rotate Q, and place the rotated K rows and the V rows into the KV cache
+    [L, S, hk, ctx, D] at each token's absolute index (the engine's keyCache /
+    valueCache of HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM
+    rides the text-only engine").  Planes: the decode form at the token's index
+    under its sequence's (start, amount).  Returns (q, k_cache, v_cache,
+    status) with status bit 2 set when a token falls outside the cache."""
+    start = np.asarray(start, np.int32)
+    amount = np.asarray(amount, np.int32)
+    n = q_bits.shape[1] if q_bits is not None else k_bits.shape[1]
+    b, p = token_index(n, start.shape[0], cu_seqlens, pos_offset)
+    pos = positions_step(p.astype(np.int32), start[b], amount[b])
+    q_out = rotate_bf16(q_bits, pos, theta, sections, rot_dim) if q_bits is not None else None
+    kc = np.array(k_cache_bits, copy=True) if k_cache_bits is not None else None
+    vc = np.array(v_cache_bits, copy=True) if v_cache_bits is not None else None
+    status = 0
+    if k_bits is not None:
+        k_rot = rotate_bf16(k_bits, pos, theta, sections, rot_dim)
+        slot = b if cache_slot is None else np.asarray(cache_slot, np.int64)[b]
+        S, ctx = kc.shape[1], kc.shape[3]
+        for t in range(n):
+            if 0 <= p[t] < ctx and 0 <= slot[t] < S:
+                kc[:, slot[t], :, p[t], :] = k_rot[:, t]
+                vc[:, slot[t], :, p[t], :] = v_bits[:, t]
+            else:
+                status |= 2
+    return q_out, kc, vc, status

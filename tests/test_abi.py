@@ -28,8 +28,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
-                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_status_string",
-                          "cmr_last_error_message", "cmr_version"}
+                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache",
+                          "cmr_status_string", "cmr_last_error_message", "cmr_version"}
     assert set(names) == set(cmr.SIGNATURES)
 
 
@@ -48,7 +48,7 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 10100
+    assert lib.cmr_version() == 10200
 
 
 SEC = (ctypes.c_int32 * 3)(11, 11, 10)
@@ -124,4 +124,17 @@ def test_rotate_shift_rejects_bad_arguments_on_the_host(lib, kw):
     a.update(kw)
     st = lib.cmr_rotate_qk_shift(a["q"], a["k"], a["cu"], a["num_seqs"], a["off"], a["start"],
                                  a["amount"], a["n"], 1, 8, 2, 256, 1e7, SEC, a["rot_dim"], None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+
+
+@pytest.mark.parametrize("kw", [
+    dict(v=None), dict(kc=None), dict(vc=None), dict(v=FAKE + 8), dict(kc=FAKE + 4),
+    dict(seqs=0), dict(ctx=0), dict(num_seqs=0), dict(start=None),
+])
+def test_rotate_cache_rejects_bad_arguments_on_the_host(lib, kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, kc=FAKE, vc=FAKE, seqs=4, ctx=64, num_seqs=2, start=FAKE)
+    a.update(kw)
+    st = lib.cmr_rotate_qk_cache(a["q"], a["k"], a["v"], FAKE, a["num_seqs"], None, a["start"],
+                                 FAKE, 10, 1, 8, 2, 256, 1e7, SEC, 64, a["kc"], a["vc"],
+                                 a["seqs"], a["ctx"], None, None, None)
     assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()

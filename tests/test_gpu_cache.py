@@ -1,0 +1,131 @@
+"""GPU parity of the fused rotate + KV-cache write, through the C ABI:
+Q rotated in place, rotated K rows and V rows placed at each token's index."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import assert_bf16_close
+from vlm_decoder_positional_b200 import cmr, inputs
+
+pytestmark = pytest.mark.gpu
+SENTINEL = 0x7F7F
+
+
+def t32(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+
+
+def bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def sentinel_cache(shape, dev):
+    return torch.full(shape, SENTINEL, dtype=torch.int16, device=dev).view(torch.bfloat16)
+
+
+def rand(shape, g, dev):
+    return torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+
+
+def run_and_compare(q, k, v, start, amount, kc, vc, cu=None, off=None, slot=None, status_want=0):
+    dev = q.device
+    q_in, k_in, v_in = bits(q), bits(k), bits(v)
+    kc_in, vc_in = bits(kc), bits(vc)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    cmr.rotate_qk_cache(q, k, v, start, amount, kc, vc, cu_seqlens=cu, pos_offset=off,
+                        cache_slot=slot, device_status=status)
+    torch.cuda.synchronize()
+    np_ = lambda t: None if t is None else t.cpu().numpy()
+    qo, kco, vco, st = oracle.rotate_qk_cache(q_in, k_in, v_in, np_(start), np_(amount), kc_in,
+                                              vc_in, np_(cu), np_(off), np_(slot))
+    assert int(status.item()) == st == status_want
+    assert_bf16_close(bits(q), qo, "q")
+    # K / V are only read
+    np.testing.assert_array_equal(bits(k), k_in)
+    np.testing.assert_array_equal(bits(v), v_in)
+    got_kc, got_vc = bits(kc), bits(vc)
+    np.testing.assert_array_equal(got_vc, vco)             # V rows are copies
+    written = kco != kc_in
+    np.testing.assert_array_equal(got_kc[~written], kco[~written])
+    assert_bf16_close(got_kc[written], kco[written], "k_cache")
+
+
+def test_prefill_varlen_into_permuted_slots(cuda_device):
+    dev = cuda_device
+    wl = inputs.make_config(2, device=dev)
+    _, s, a = cmr.positions(t32(wl.ids, dev), t32(wl.cu_seqlens, dev))
+    g = torch.Generator(device=dev).manual_seed(1)
+    n = wl.n_tokens
+    v = rand((1, n, 2, 256), g, dev)
+    S, ctx = 20, 520
+    kc = sentinel_cache((1, S, 2, ctx, 256), dev)
+    vc = sentinel_cache((1, S, 2, ctx, 256), dev)
+    slot = t32(np.random.default_rng(3).permutation(S)[:wl.num_seqs], dev)
+    run_and_compare(wl.q, wl.k, v, s, a, kc, vc, cu=t32(wl.cu_seqlens, dev), slot=slot)
+
+
+def test_decode_appends_at_each_sequences_length(cuda_device):
+    dev = cuda_device
+    rng = np.random.default_rng(4)
+    B, ctx = 64, 4096                        # the engine's context limit
+    prior = rng.integers(73, ctx, size=B)
+    origins = np.array([rng.integers(0, p_ - 67 + 1) for p_ in prior])
+    wl = inputs.make_batch(prior, origins, with_qk=False, device=dev)
+    _, s, a = cmr.positions(t32(wl.ids, dev), t32(wl.cu_seqlens, dev))
+    g = torch.Generator(device=dev).manual_seed(5)
+    L = 2
+    q, k, v = rand((L, B, 8, 256), g, dev), rand((L, B, 2, 256), g, dev), rand((L, B, 2, 256), g, dev)
+    kc = sentinel_cache((L, B, 2, ctx, 256), dev)
+    vc = sentinel_cache((L, B, 2, ctx, 256), dev)
+    run_and_compare(q, k, v, s, a, kc, vc, off=t32(prior, dev))
+
+
+def test_out_of_range_tokens_write_nothing_and_flag(cuda_device):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(6)
+    B = 5
+    q, k, v = rand((2, B, 4, 128), g, dev), rand((2, B, 3, 128), g, dev), rand((2, B, 3, 128), g, dev)
+    kc = sentinel_cache((2, 3, 3, 16, 128), dev)
+    vc = sentinel_cache((2, 3, 3, 16, 128), dev)
+    start = t32([1 << 30] * B, dev)
+    amount = t32([0] * B, dev)
+    off = t32([0, 15, 16, 3, -1], dev)       # 16 and -1 fall outside ctx 16
+    slot = t32([0, 1, 2, 5, 1], dev)         # slot 5 falls outside S 3
+    run_and_compare(q, k, v, start, amount, kc, vc, off=off, slot=slot,
+                    status_want=cmr.CMR_DEVICE_CACHE_RANGE)
+
+
+def test_q_only_needs_no_cache(cuda_device):
+    dev = cuda_device
+    g = torch.Generator(device=dev).manual_seed(7)
+    q = rand((1, 40, 8, 256), g, dev)
+    q_in = bits(q)
+    start, amount = t32([73], dev), t32([58], dev)
+    cmr.rotate_qk_cache(q, None, None, start, amount, None, None, cu_seqlens=t32([0, 40], dev),
+                        pos_offset=t32([50], dev))
+    torch.cuda.synchronize()
+    p = oracle.positions_step(np.arange(50, 90), np.full(40, 73), np.full(40, 58))
+    assert_bf16_close(bits(q), oracle.rotate_bf16(q_in, p), "q")
+
+
+def test_cache_path_matches_shift_path_bit_for_bit(cuda_device):
+    # Q after the cache form equals Q after cmr_rotate_qk_shift, and the cached
+    # K rows equal K rotated in place by cmr_rotate_qk_shift.
+    dev = cuda_device
+    wl = inputs.make_config(3, device=dev)
+    cu = t32(wl.cu_seqlens, dev)
+    _, s, a = cmr.positions(t32(wl.ids, dev), cu)
+    v = wl.k.clone()
+    kc = sentinel_cache((1, 64, 2, 4096, 256), dev)
+    vc = sentinel_cache((1, 64, 2, 4096, 256), dev)
+    q2, k2 = wl.q.clone(), wl.k.clone()
+    cmr.rotate_qk_cache(wl.q, wl.k, v, s, a, kc, vc, cu_seqlens=cu)
+    cmr.rotate_qk_shift(q2, k2, s, a, cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert torch.equal(wl.q.view(torch.int16), q2.view(torch.int16))
+    # prompt b's tokens fill cache rows [b, :, 0:4096] in order
+    kc_tokens = kc.view(1, 64, 2, 4096, 256).permute(0, 1, 3, 2, 4).reshape(1, 64 * 4096, 2, 256)
+    assert torch.equal(kc_tokens.view(torch.int16), k2.view(torch.int16))
+    vc_tokens = vc.permute(0, 1, 3, 2, 4).reshape(1, 64 * 4096, 2, 256)
+    assert torch.equal(vc_tokens.view(torch.int16), v.view(torch.int16))

@@ -182,3 +182,32 @@ def test_bf16_output_is_correctly_rounded_f64():
     pos = np.random.default_rng(8).integers(0, 30000, size=(3, 64)).astype(np.int32)
     y, f64 = oracle.rotate_bf16(x, pos, return_f64=True)
     np.testing.assert_array_equal(y[..., :64], oracle.f64_to_bf16(f64[..., :64]))
+
+
+def test_cache_form_places_rotated_rows_at_each_tokens_index():
+    # the cache form composes the pinned pieces: planes of the decode form at
+    # the token's index, the pinned rotation, and a placement at [l, slot, h, p]
+    L, n, hk, D = 2, 9, 2, 128
+    q = rand_bf16((L, n, 3, D), 30)
+    k = rand_bf16((L, n, hk, D), 31)
+    v = rand_bf16((L, n, hk, D), 32)
+    cu = np.array([0, 4, 4, 9], np.int32)               # an empty middle sequence
+    off = np.array([70, 0, 3], np.int32)
+    start = np.array([73, 1 << 30, 10], np.int32)
+    amount = np.array([58, 0, 1], np.int32)
+    slot = np.array([2, 0, 1], np.int32)
+    kc0 = np.full((L, 3, hk, 8, D), 0x7F7F, np.uint16)
+    vc0 = np.full((L, 3, hk, 8, D), 0x7F7F, np.uint16)
+    qo, kc, vc, status = oracle.rotate_qk_cache(q, k, v, start, amount, kc0, vc0, cu, off, slot)
+    assert status == 2                                  # sequence 0 sits at 70..73 > ctx 8
+    p = np.array([70, 71, 72, 73, 3, 4, 5, 6, 7])
+    b = np.array([0, 0, 0, 0, 2, 2, 2, 2, 2])
+    pos = oracle.positions_step(p, start[b], amount[b])
+    np.testing.assert_array_equal(qo, oracle.rotate_bf16(q, pos))
+    kr = oracle.rotate_bf16(k, pos)
+    written = np.zeros(kc0.shape[:4], bool)
+    for t in range(4, 9):
+        np.testing.assert_array_equal(kc[:, 1, :, p[t]], kr[:, t])
+        np.testing.assert_array_equal(vc[:, 1, :, p[t]], v[:, t])
+        written[:, 1, :, p[t]] = True
+    assert (kc[~written] == 0x7F7F).all() and (vc[~written] == 0x7F7F).all()

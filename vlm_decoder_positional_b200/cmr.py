@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libcmr.so")
 
 CMR_OK, CMR_EINVAL, CMR_ECUDA, CMR_EUNSUPPORTED = 0, 1, 2, 3
 CMR_DEVICE_BAD_CU_SEQLENS = 1
+CMR_DEVICE_CACHE_RANGE = 2
 RULES = {"canvas": 0, "qwen_vl": 1, "planes_1d": 2}
 TEXT_ONLY_START = 1 << 30
 
@@ -37,6 +38,13 @@ SIGNATURES = {
                                            ctypes.c_int32, ctypes.c_double,
                                            ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
                                            ctypes.c_void_p]),
+    "cmr_rotate_qk_cache": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           _i32p, ctypes.c_int32, _i32p, _i32p, _i32p,
+                                           ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                           ctypes.c_int32, _i32p, _i32p, ctypes.c_void_p]),
     "cmr_rotate_qk": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p, ctypes.c_int64,
                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.c_double,
@@ -273,6 +281,68 @@ def rotate_qk_shift(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
             start.data_ptr() if b else None, amount.data_ptr() if b else None, n, L, hq, hk, D,
             float(theta), sec, int(rot_dim), _stream_ptr(dev, stream)), "cmr_rotate_qk_shift")
     return q, k
+
+
+def rotate_qk_cache(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                    v: Optional[torch.Tensor], start: torch.Tensor, amount: torch.Tensor,
+                    k_cache: Optional[torch.Tensor], v_cache: Optional[torch.Tensor],
+                    cu_seqlens: Optional[torch.Tensor] = None,
+                    pos_offset: Optional[torch.Tensor] = None,
+                    cache_slot: Optional[torch.Tensor] = None, theta: float = 1e7,
+                    sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
+                    device_status: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None):
+    """cmr_rotate_qk_cache: rotate q in place and write the rotated k rows and
+    the v rows into k_cache / v_cache [L, S, hk, ctx, D] at each token's index.
+    Returns q."""
+    _want(start, "start", torch.int32)
+    dev = start.device
+    _want(amount, "amount", torch.int32, dev)
+    b = start.numel()
+    ref = q if q is not None else k
+    n = ref.shape[-3] if ref is not None else 0
+    L, hq, hk, D = _qk_shapes(q, k, dev, n)
+    if hk:
+        if v is None or k_cache is None or v_cache is None:
+            raise ValueError("v, k_cache and v_cache are required with K heads")
+        _qk_shapes(None, v, dev, n)
+        if tuple(v.shape[-2:]) != (hk, D):
+            raise ValueError("v must have the shape of k")
+        for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+            _want(t, name, torch.bfloat16, dev)
+            if t.dim() != 5 or t.shape[0] != L or t.shape[2] != hk or t.shape[4] != D:
+                raise ValueError(f"{name} must be [L, S, hk, ctx, D] = [{L}, S, {hk}, ctx, {D}]")
+        if k_cache.shape != v_cache.shape:
+            raise ValueError("k_cache and v_cache must have the same shape")
+        S, ctx = k_cache.shape[1], k_cache.shape[3]
+    else:
+        S = ctx = 0
+    opt = {}
+    for t, name, want_n in ((cu_seqlens, "cu_seqlens", b + 1), (pos_offset, "pos_offset", b),
+                            (cache_slot, "cache_slot", b)):
+        if t is not None:
+            _want(t, name, torch.int32, dev)
+            if t.numel() != want_n:
+                raise ValueError(f"{name} needs {want_n} entries")
+            opt[name] = t.data_ptr()
+        else:
+            opt[name] = None
+    st_ptr = None
+    if device_status is not None:
+        _want(device_status, "device_status", torch.int32, dev)
+        st_ptr = device_status.data_ptr()
+    sec = (ctypes.c_int32 * 3)(*[int(x) for x in sections])
+
+    def ptr(t):
+        return t.data_ptr() if t is not None and t.numel() else None
+
+    with torch.cuda.device(dev):
+        _check(lib().cmr_rotate_qk_cache(
+            ptr(q), ptr(k), ptr(v), opt["cu_seqlens"], b, opt["pos_offset"],
+            start.data_ptr() if b else None, amount.data_ptr() if b else None, n, L, hq, hk, D,
+            float(theta), sec, int(rot_dim), ptr(k_cache), ptr(v_cache), S, ctx,
+            opt["cache_slot"], st_ptr, _stream_ptr(dev, stream)), "cmr_rotate_qk_cache")
+    return q
 
 
 def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor,

@@ -127,7 +127,7 @@ const char* cmr_status_string(cmr_status s) {
 
 const char* cmr_last_error_message(void) { return g_message; }
 
-int32_t cmr_version(void) { return 10100; }  // 1.1.0
+int32_t cmr_version(void) { return 10200; }  // 1.2.0
 
 cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
@@ -262,6 +262,55 @@ cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens, int3
   a.amount = amount;
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk_shift launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                               int32_t num_seqs, const int32_t* pos_offset, const int32_t* start,
+                               const int32_t* amount, int64_t n_tokens, int32_t num_layers,
+                               int32_t hq, int32_t hk, int32_t head_dim, double theta,
+                               const int32_t sections[3], int32_t rot_dim, void* k_cache,
+                               void* v_cache, int32_t cache_seqs, int32_t cache_ctx,
+                               const int32_t* cache_slot, int32_t* device_status,
+                               cmr_stream_t stream) {
+  cmr::CacheArgs ca{};
+  cmr::FreqTable table;
+  cmr_status s = check_rotate(q, const_cast<void*>(k), n_tokens, num_layers, hq, hk, head_dim,
+                              theta, sections, rot_dim, &ca.r, &table);
+  if (s != CMR_OK || ca.r.n_tokens == 0) return s;
+  if (num_seqs <= 0) return fail(CMR_EINVAL, "num_seqs must be > 0 when there are tokens");
+  if (!cu_seqlens && num_seqs != n_tokens)
+    return fail(CMR_EINVAL, "without cu_seqlens every sequence holds one token (num_seqs == n_tokens)");
+  if (!start || !amount) return fail(CMR_EINVAL, "start and amount are required");
+  if (hk > 0) {
+    if (!v || !k_cache || !v_cache) return fail(CMR_EINVAL, "v, k_cache and v_cache are required");
+    if (!aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+      return fail(CMR_EINVAL, "v, k_cache and v_cache must be 16-byte aligned");
+    if (cache_seqs <= 0 || cache_ctx <= 0) return fail(CMR_EINVAL, "cache sizes must be > 0");
+    if ((s = check_device_ptr(v, "v")) != CMR_OK) return s;
+    if ((s = check_device_ptr(k_cache, "k_cache")) != CMR_OK) return s;
+    if ((s = check_device_ptr(v_cache, "v_cache")) != CMR_OK) return s;
+  }
+  if (cu_seqlens && (s = check_device_ptr(cu_seqlens, "cu_seqlens")) != CMR_OK) return s;
+  if (pos_offset && (s = check_device_ptr(pos_offset, "pos_offset")) != CMR_OK) return s;
+  if (cache_slot && (s = check_device_ptr(cache_slot, "cache_slot")) != CMR_OK) return s;
+  if ((s = check_device_ptr(start, "start")) != CMR_OK) return s;
+  if ((s = check_device_ptr(amount, "amount")) != CMR_OK) return s;
+  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  ca.r.cu = cu_seqlens;
+  ca.r.num_seqs = num_seqs;
+  ca.r.pos_offset = pos_offset;
+  ca.r.start = start;
+  ca.r.amount = amount;
+  ca.v = static_cast<const uint16_t*>(v);
+  ca.k_cache = static_cast<uint16_t*>(k_cache);
+  ca.v_cache = static_cast<uint16_t*>(v_cache);
+  ca.cache_slot = cache_slot;
+  ca.cache_seqs = cache_seqs;
+  ca.cache_ctx = cache_ctx;
+  ca.status = device_status;
+  cudaError_t e = cmr::launch_rotate_qk_cache(ca, table, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_qk_cache launch");
   return CMR_OK;
 }
 

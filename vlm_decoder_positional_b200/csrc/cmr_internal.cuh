@@ -42,9 +42,29 @@ struct RotateArgs {
   int32_t num_layers;
   int32_t hq, hk, head_dim, rot_dim;
   int32_t units_per_head;  // rot_dim / 16: threads per token, 8 frequencies each
-  int32_t head_groups;      // work items per token (set at launch)
-  int32_t heads_per_group;
+  int32_t job_groups;       // work items per token (set at launch)
+  int32_t jobs_per_group;   // (layer, head) rows per work item
 };
+
+// Rotate Q in place and write rotated K and V rows into a KV cache
+// [num_layers, cache_seqs, hk, cache_ctx, head_dim]; planes from the shift state.
+struct CacheArgs {
+  RotateArgs r;           // q, k (read only here), shift state, shape
+  const uint16_t* v;      // bf16 bits [L, N, hk, D]
+  uint16_t* k_cache;
+  uint16_t* v_cache;
+  const int32_t* cache_slot;  // [num_seqs] cache row of each sequence, or nullptr: b
+  int32_t cache_seqs;
+  int32_t cache_ctx;
+  int32_t* status;        // optional device status word
+  // work split (set at launch): Q rows and KV rows of a token form separate
+  // items, each split into groups of (layer, head) rows
+  int32_t q_groups, q_rows_per_group;
+  int32_t kv_groups, kv_rows_per_group;
+};
+
+cudaError_t launch_rotate_qk_cache(const CacheArgs& args, const FreqTable& table,
+                                   cudaStream_t stream);
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                              int64_t n_tokens, int32_t image_token_id, int32_t rule,
