@@ -1,0 +1,43 @@
+"""The host-buffer pipeline gives exactly the device path's results."""
+import numpy as np
+import pytest
+import torch
+
+from vlm_decoder_positional_b200 import cmr, inputs, pipeline
+
+pytestmark = pytest.mark.gpu
+
+
+def test_prompt_chunks_cover_the_batch():
+    cu = np.array([0, 5, 5, 30, 31, 100, 101], np.int64)
+    ch = pipeline.prompt_chunks(cu, 30)
+    assert ch[0][0] == 0 and ch[-1][1] == 6
+    assert all(a[1] == b[0] for a, b in zip(ch, ch[1:]))
+    assert all(cu[s1] - cu[s0] <= 30 or s1 - s0 == 1 for s0, s1 in ch)
+
+
+@pytest.mark.parametrize("cfg,chunk", [(2, 1000), (3, 3 * 4096), (5, 2 * 8192)])
+def test_host_pipeline_matches_the_device_path(cuda_device, cfg, chunk):
+    wl = inputs.make_config(cfg, device=cuda_device)
+    dev = cuda_device
+    ref_q, ref_k = wl.q.clone(), wl.k.clone()
+    pos, s, a = cmr.positions(torch.from_numpy(wl.ids).to(dev), torch.from_numpy(wl.cu_seqlens).to(dev))
+    cmr.rotate_qk(ref_q, ref_k, pos)
+    q_h = wl.q.cpu().pin_memory()
+    k_h = wl.k.cpu().pin_memory()
+    ids_h = torch.from_numpy(wl.ids).pin_memory()
+    pos_h = torch.empty((3, wl.n_tokens), dtype=torch.int32, pin_memory=True)
+    st_h = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
+    am_h = torch.empty(wl.num_seqs, dtype=torch.int32, pin_memory=True)
+    lens = np.diff(wl.cu_seqlens)
+    pl = pipeline.HostPipeline(dev, wl.num_layers, wl.hq, wl.hk, wl.head_dim,
+                               max_chunk_tokens=max(chunk, int(lens.max())),
+                               max_chunk_seqs=wl.num_seqs, depth=3)
+    for _ in range(2):   # the second run reuses the ring (inputs rotated twice)
+        pl.run(ids_h, wl.cu_seqlens, q_h, k_h, pos_h, st_h, am_h, chunk_tokens=chunk)
+    torch.cuda.synchronize()
+    cmr.rotate_qk(ref_q, ref_k, pos)
+    torch.cuda.synchronize()
+    assert torch.equal(pos_h, pos.cpu()) and torch.equal(st_h, s.cpu()) and torch.equal(am_h, a.cpu())
+    assert torch.equal(q_h.view(torch.int16), ref_q.cpu().view(torch.int16))
+    assert torch.equal(k_h.view(torch.int16), ref_k.cpu().view(torch.int16))
