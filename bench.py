@@ -156,10 +156,19 @@ class ClockSampler:
 # CPU side: the oracle on a bounded sample (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl_cpu, n):
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(wl_cpu, n, threads=1):
     """One oracle pass over a sample: the planes of the prompts that hold the
     first n tokens (decode: of the first n prompts, then their new token),
-    then the rotation of those n tokens' Q/K rows, every layer and head."""
+    then the rotation of those n tokens' Q/K rows, every layer and head.  With
+    threads > 1 the rotation's token range is split over a thread pool (the
+    oracle is C called through ctypes, which releases the GIL)."""
     import oracle
     cu = wl_cpu["cu"]
     if wl_cpu["cache_len"] is None:
@@ -170,8 +179,19 @@ def oracle_sample_step(wl_cpu, n):
         _, start, amount = oracle.positions(wl_cpu["ids"][: cu[n]], cu[: n + 1],
                                             inputs.IMAGE_TOKEN_ID)
         pos = oracle.positions_step(wl_cpu["cache_len"][:n], start, amount)
-    oracle.rotate_bf16(wl_cpu["q"][:, :n], pos)
-    oracle.rotate_bf16(wl_cpu["k"][:, :n], pos)
+
+    def rotate(lo, hi):
+        p = np.ascontiguousarray(pos[:, lo:hi])
+        oracle.rotate_bf16(wl_cpu["q"][:, lo:hi], p)
+        oracle.rotate_bf16(wl_cpu["k"][:, lo:hi], p)
+
+    if threads <= 1:
+        rotate(0, n)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        cuts = np.linspace(0, n, threads + 1).astype(int)
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(lambda i: rotate(cuts[i], cuts[i + 1]), range(threads)))
     return n
 
 
@@ -182,34 +202,46 @@ def cpu_sample_inputs(wl, n_max):
             "cache_len": wl.cache_len}
 
 
-def calibrate_sample(wl_cpu, seconds, n_max):
-    """Tokens whose oracle pass takes about `seconds` on this host (at most n_max)."""
-    probe = min(256, n_max)
+def calibrate_sample(wl_cpu, seconds, n_max, threads=1):
+    """Tokens whose oracle pass takes about `seconds` on this host (at most n_max),
+    estimated from a probe on the tokens wl_cpu holds."""
+    probe = min(256 * threads, n_max, wl_cpu["q"].shape[1])
     t0 = time.perf_counter()
-    oracle_sample_step(wl_cpu, probe)
+    oracle_sample_step(wl_cpu, probe, threads)
     dt = time.perf_counter() - t0
     return int(max(probe, min(n_max, probe * seconds / max(dt, 1e-6))))
 
 
-def sample_label(wl, n):
+def sample_label(wl, n, threads=1):
+    tail = f"fp64, {threads} thread{'s' if threads > 1 else ''}"
     if wl.cache_len is not None:
         return (f"planes of the first {n} prompts + their new token, rotation of those {n} "
-                f"tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
+                f"tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, {tail}")
     b = int(np.searchsorted(wl.cu_seqlens, n, side="left"))
     return (f"planes of the first {b} prompts ({wl.cu_seqlens[b]} tokens) + rotation of the "
-            f"first {n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, fp64, 1 thread")
+            f"first {n} tokens x {wl.num_layers} layers x {wl.hq + wl.hk} heads, {tail}")
 
 
 def run_cpu_baseline(wl, seconds):
-    # size the copy to the host from a quick estimate, then calibrate on it
-    n_max = min(wl.qk_tokens, 200_000)
-    wl_cpu = cpu_sample_inputs(wl, n_max)
-    n = calibrate_sample(wl_cpu, seconds, n_max)
-    t0 = time.perf_counter()
-    oracle_sample_step(wl_cpu, n)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": sample_label(wl, n) + f", {dt:.1f} s"}
+    """The oracle on all host cores (and on one, for reference) over a bounded
+    sample of the workload, about `seconds` of work each."""
+    cores = host_cores()
+    n_cap = min(wl.qk_tokens, 200_000)
+    probe_inputs = cpu_sample_inputs(wl, min(n_cap, 256 * cores))
+    out = {}
+    for threads in sorted({1, cores}, reverse=True):
+        n = calibrate_sample(probe_inputs, seconds, n_cap, threads)
+        wl_cpu = cpu_sample_inputs(wl, n) if n > probe_inputs["q"].shape[1] else probe_inputs
+        t0 = time.perf_counter()
+        oracle_sample_step(wl_cpu, n, threads)
+        dt = time.perf_counter() - t0
+        out[threads] = (n / dt, sample_label(wl, n, threads) + f", {dt:.1f} s")
+        del wl_cpu
+    value, sample = out[cores]
+    res = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    if cores > 1:
+        res["single_thread"] = {"value": out[1][0], "sample": out[1][1]}
+    return res
 
 
 def run_reference(args):
@@ -218,28 +250,30 @@ def run_reference(args):
         return 0
     # the same prompts (ids); Q/K drawn only for the sampled tokens
     wl = inputs.make_config(args.workload, device="cpu", with_qk=False)
+    cores = host_cores()
     per_step = max(1.0, args.reference_budget_s / (args.steps + args.warmup))
-    n_max = min(wl.num_seqs if wl.cache_len is not None else wl.n_tokens, 65_536)
+    n_max = min(wl.num_seqs if wl.cache_len is not None else wl.n_tokens, 200_000)
     wl.q = inputs.random_qk((wl.num_layers, n_max, wl.hq, wl.head_dim), wl.seed + 1)
     wl.k = inputs.random_qk((wl.num_layers, n_max, wl.hk, wl.head_dim), wl.seed + 2)
     wl_cpu = cpu_sample_inputs(wl, n_max)
-    n = calibrate_sample(wl_cpu, per_step, n_max)
+    n = calibrate_sample(wl_cpu, per_step, n_max, cores)
     for _ in range(args.warmup):
-        oracle_sample_step(wl_cpu, n)
+        oracle_sample_step(wl_cpu, n, cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_sample_step(wl_cpu, n)
+        oracle_sample_step(wl_cpu, n, cores)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
-    sample = "per step: " + sample_label(wl, n)
+    sample = "per step: " + sample_label(wl, n, cores)
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": {"workload": workload_label(wl), "global_batch": wl.n_tokens,
-                   "seq_len": wl.n_tokens // wl.num_seqs, "parallelism": "cpu oracle, 1 thread"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "seq_len": wl.n_tokens // wl.num_seqs,
+                   "parallelism": f"cpu oracle, {cores} threads"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -1,0 +1,45 @@
+"""bench.py's host-side pieces: algorithmic byte counts, the traffic record,
+and the reference (oracle) arm's JSON line, all on CPU."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+from vlm_decoder_positional_b200 import inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_match_the_hand_count():
+    # 2,560 B per token-layer for 8 Q + 2 K heads x 64 dims x bf16 x (read + write)
+    assert bench.rotate_bytes(1, 1, 8, 2, 64) == 2560 + 12
+    assert bench.rotate_bytes(262144, 6, 8, 2, 64) == 4_026_531_840 + 3_145_728
+    assert bench.positions_bytes(262144, 32) == 262144 * 16 + 32 * 12
+
+
+def test_traffic_record_is_tied_to_the_kernel_source_and_workload():
+    t = bench.recorded_traffic("c5_6layers_32x8192")
+    assert t is None or 3.5e9 < t < 4.5e9
+    assert bench.recorded_traffic("some_other_workload") is None
+
+
+def test_oracle_sample_step_threads_agree():
+    wl = inputs.make_config(2)
+    wl_cpu = bench.cpu_sample_inputs(wl, 600)
+    assert bench.oracle_sample_step(wl_cpu, 600, threads=1) == 600
+    assert bench.oracle_sample_step(wl_cpu, 600, threads=4) == 600
+    assert "16 prompts" not in bench.sample_label(wl, 600)
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "1",
+                          "--steps", "3", "--warmup", "3", "--reference-budget-s", "2"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=300, check=True)
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
