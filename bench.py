@@ -503,14 +503,17 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
         h2d = h_q.numel() * 2 + h_k.numel() * 2 + 12 * wl.num_seqs
         d2h = h_q.numel() * 2 + h_k.numel() * 2
     else:
-        h2d = h_ids.numel() * 4 + h_cu.numel() * 4 + h_q.numel() * 2 + h_k.numel() * 2
-        d2h = h_q.numel() * 2 + h_k.numel() * 2 + h_pos.numel() * 4 + 8 * wl.num_seqs
+        # the pipeline moves only the rotated dims of every head row
+        rot = (h_q.numel() + h_k.numel()) // wl.head_dim * wl.rot_dim * 2
+        h2d = h_ids.numel() * 4 + h_cu.numel() * 4 + rot
+        d2h = rot + h_pos.numel() * 4 + 8 * wl.num_seqs
     return {"value": tokens_all * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
             "path": ("pinned host -> cmr.rotate_qk_shift -> pinned host" if decode else
-                     "pinned host -> HostPipeline: chunks of whole prompts, copies in, "
-                     "cmr.positions + cmr.rotate_qk, copies out on three streams -> pinned host")}
+                     "pinned host -> HostPipeline: chunks of whole prompts, rotated dims in "
+                     "(pitched copies), cmr.positions + cmr.rotate_qk, rotated dims out, on "
+                     "three streams -> pinned host")}
 
 
 def main():

@@ -244,6 +244,22 @@ CMR_API cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v,
                                        int32_t cache_ctx, const int32_t* cache_slot,
                                        int32_t* device_status, cmr_stream_t stream);
 
+/* Copy only the rotated dims of head rows between host and device memory: the
+ * first rot_dim of every head_dim-wide bf16 row (a pitched copy of rot_dim * 2
+ * bytes out of every head_dim * 2), for `rows` consecutive rows, on `stream`.
+ * For callers whose Q/K live in host memory: the rotation reads and writes
+ * only these dims, so moving the rest over PCIe is wasted; rows copied back
+ * keep their untouched dims on the host side.
+ *
+ *   dst, src    host (pinned for asynchrony) or device memory, one of each
+ *   rows        >= 0 rows of head_dim bf16 elements each
+ *   direction   0: host -> device, 1: device -> host
+ * Errors: CMR_EINVAL for null pointers, rot_dim > head_dim or non-positive
+ * sizes, an unknown direction; CMR_ECUDA if the copy cannot be enqueued. */
+CMR_API cmr_status cmr_copy_rotated_dims(void* dst, const void* src, int64_t rows,
+                                         int32_t head_dim, int32_t rot_dim,
+                                         int32_t direction, cmr_stream_t stream);
+
 /* Static, never-null description of a status code. */
 CMR_API const char* cmr_status_string(cmr_status s);
 

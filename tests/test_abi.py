@@ -29,7 +29,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
                           "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache",
-                          "cmr_status_string", "cmr_last_error_message", "cmr_version"}
+                          "cmr_copy_rotated_dims", "cmr_status_string",
+                          "cmr_last_error_message", "cmr_version"}
     assert set(names) == set(cmr.SIGNATURES)
 
 
@@ -48,7 +49,7 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 10200
+    assert lib.cmr_version() == 10300
 
 
 SEC = (ctypes.c_int32 * 3)(11, 11, 10)
@@ -138,3 +139,15 @@ def test_rotate_cache_rejects_bad_arguments_on_the_host(lib, kw):
                                  FAKE, 10, 1, 8, 2, 256, 1e7, SEC, 64, a["kc"], a["vc"],
                                  a["seqs"], a["ctx"], None, None, None)
     assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+
+
+@pytest.mark.parametrize("args", [
+    (FAKE, FAKE, -1, 256, 64, 0), (FAKE, FAKE, 10, 64, 128, 0), (FAKE, FAKE, 10, 256, 64, 2),
+    (None, FAKE, 10, 256, 64, 0), (FAKE, None, 10, 256, 64, 1), (FAKE, FAKE, 10, 0, 0, 0),
+])
+def test_copy_rotated_dims_rejects_bad_arguments(lib, args):
+    assert lib.cmr_copy_rotated_dims(*args, None) == cmr.CMR_EINVAL
+
+
+def test_copy_rotated_dims_of_nothing_is_a_no_op(lib):
+    assert lib.cmr_copy_rotated_dims(None, None, 0, 256, 64, 0, None) == cmr.CMR_OK

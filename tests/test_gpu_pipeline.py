@@ -41,3 +41,17 @@ def test_host_pipeline_matches_the_device_path(cuda_device, cfg, chunk):
     assert torch.equal(pos_h, pos.cpu()) and torch.equal(st_h, s.cpu()) and torch.equal(am_h, a.cpu())
     assert torch.equal(q_h.view(torch.int16), ref_q.cpu().view(torch.int16))
     assert torch.equal(k_h.view(torch.int16), ref_k.cpu().view(torch.int16))
+
+
+def test_copy_rotated_dims_moves_exactly_the_rotated_dims(cuda_device):
+    g = torch.Generator().manual_seed(1)
+    h = torch.randn((3, 50, 4, 256), generator=g).to(torch.bfloat16).pin_memory()
+    d = torch.full((3, 50, 4, 256), 7.0, dtype=torch.bfloat16, device=cuda_device)
+    cmr.copy_rotated_dims(d, h, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(d[..., :64].cpu(), h[..., :64])
+    assert (d[..., 64:] == 7.0).all()
+    back = torch.zeros_like(h).pin_memory()
+    cmr.copy_rotated_dims(back, d, 64)
+    torch.cuda.synchronize()
+    assert torch.equal(back[..., :64], h[..., :64]) and (back[..., 64:] == 0).all()

@@ -50,6 +50,9 @@ SIGNATURES = {
                                      ctypes.c_int32, ctypes.c_double,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
                                      ctypes.c_void_p]),
+    "cmr_copy_rotated_dims": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_void_p]),
     "cmr_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cmr_last_error_message": (ctypes.c_char_p, []),
     "cmr_version": (ctypes.c_int32, []),
@@ -364,3 +367,25 @@ def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.T
                                    sec, int(rot_dim), _stream_ptr(dev, stream)),
                "cmr_rotate_qk")
     return q, k
+
+
+def copy_rotated_dims(dst: torch.Tensor, src: torch.Tensor, rot_dim: int = 64,
+                      stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """cmr_copy_rotated_dims: copy dims [0, rot_dim) of every head row of a bf16
+    tensor [..., head_dim] between host (pinned) and device memory."""
+    for t, name in ((dst, "dst"), (src, "src")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor")
+    if dst.shape != src.shape:
+        raise ValueError("dst and src must have the same shape")
+    if dst.is_cuda == src.is_cuda:
+        raise ValueError("one of dst, src must be on the GPU and the other on the host")
+    dev = dst.device if dst.is_cuda else src.device
+    head_dim = dst.shape[-1]
+    rows = dst.numel() // head_dim if head_dim else 0
+    with torch.cuda.device(dev):
+        _check(lib().cmr_copy_rotated_dims(dst.data_ptr() if rows else None,
+                                           src.data_ptr() if rows else None, rows, head_dim,
+                                           int(rot_dim), 0 if dst.is_cuda else 1,
+                                           _stream_ptr(dev, stream)), "cmr_copy_rotated_dims")
+    return dst

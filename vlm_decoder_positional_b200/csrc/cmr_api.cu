@@ -127,7 +127,7 @@ const char* cmr_status_string(cmr_status s) {
 
 const char* cmr_last_error_message(void) { return g_message; }
 
-int32_t cmr_version(void) { return 10200; }  // 1.2.0
+int32_t cmr_version(void) { return 10300; }  // 1.3.0
 
 cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
@@ -311,6 +311,22 @@ cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v, const int3
   ca.status = device_status;
   cudaError_t e = cmr::launch_rotate_qk_cache(ca, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk_cache launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_copy_rotated_dims(void* dst, const void* src, int64_t rows, int32_t head_dim,
+                                 int32_t rot_dim, int32_t direction, cmr_stream_t stream) {
+  if (rows < 0 || head_dim <= 0 || rot_dim <= 0 || rot_dim > head_dim)
+    return fail(CMR_EINVAL, "need rows >= 0 and 0 < rot_dim <= head_dim");
+  if (direction != 0 && direction != 1) return fail(CMR_EINVAL, "direction must be 0 or 1");
+  if (rows == 0) return CMR_OK;
+  if (!dst || !src) return fail(CMR_EINVAL, "dst and src are required");
+  const size_t pitch = static_cast<size_t>(head_dim) * 2;
+  const size_t width = static_cast<size_t>(rot_dim) * 2;
+  cudaError_t e = cudaMemcpy2DAsync(dst, pitch, src, pitch, width, static_cast<size_t>(rows),
+                                    direction == 0 ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy2DAsync");
   return CMR_OK;
 }
 

@@ -6,8 +6,10 @@ need nothing from another chunk).  Each chunk goes host -> device on one stream,
 through cmr_positions + cmr_rotate_qk on a second, and back on a third, over a
 ring of `depth` device buffers, so the host-to-device copy of one chunk, the
 kernels of the next and the device-to-host copy of a third run at the same
-time (PCIe moves both directions at once).  Only copies, streams and events
-live here; every step of the method runs in the library's kernels.
+time (PCIe moves both directions at once).  Only the rotated dims of each head
+row cross PCIe (cmr_copy_rotated_dims, a pitched copy): the rest of Q/K is
+neither read nor written by the method.  Only copies, streams and events live
+here; every step of the method runs in the library's kernels.
 """
 from typing import List, Tuple
 
@@ -97,9 +99,9 @@ class HostPipeline:
                     self.s_in.wait_event(self.copied_out[r])  # ring slot free again
                 self.cu[r][:b + 1].copy_(self.cu_stage[r][:b + 1], non_blocking=True)
                 self.ids[r][:n].copy_(ids_host[t0:t1], non_blocking=True)
-                for l in range(L):
-                    q_d[l].copy_(q_host[l, t0:t1], non_blocking=True)
-                    k_d[l].copy_(k_host[l, t0:t1], non_blocking=True)
+                for l in range(L):  # only the rotated dims of each head row
+                    cmr.copy_rotated_dims(q_d[l], q_host[l, t0:t1], rot_dim, self.s_in)
+                    cmr.copy_rotated_dims(k_d[l], k_host[l, t0:t1], rot_dim, self.s_in)
                 self.copied_in[r].record(self.s_in)
             with torch.cuda.stream(self.s_run):
                 self.s_run.wait_event(self.copied_in[r])
@@ -110,8 +112,8 @@ class HostPipeline:
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(self.computed[r])
                 for l in range(L):
-                    q_host[l, t0:t1].copy_(q_d[l], non_blocking=True)
-                    k_host[l, t0:t1].copy_(k_d[l], non_blocking=True)
+                    cmr.copy_rotated_dims(q_host[l, t0:t1], q_d[l], rot_dim, self.s_out)
+                    cmr.copy_rotated_dims(k_host[l, t0:t1], k_d[l], rot_dim, self.s_out)
                 for plane in range(3):
                     pos_host[plane, t0:t1].copy_(pos_d[plane], non_blocking=True)
                 start_host[s0:s1].copy_(self.start[r][:b], non_blocking=True)
