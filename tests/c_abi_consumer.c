@@ -1,0 +1,91 @@
+/* A plain C11 consumer of the C ABI (include/cmr.h), used by
+ * tests/test_c_consumer.py.
+ *   ./consumer host    -- version, status strings and host-side argument
+ *                         checks; never touches a GPU
+ *   ./consumer device  -- the planes of one 80-token prompt with <image> at
+ *                         index 6, in cudaMalloc'd buffers; prints "p T H W"
+ *                         lines and "start amount" for the test to compare */
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "cmr.h"
+
+#define CHECK(cond)                                             \
+  do {                                                          \
+    if (!(cond)) {                                              \
+      fprintf(stderr, "check failed: %s (line %d)\n", #cond, __LINE__); \
+      return 1;                                                 \
+    }                                                           \
+  } while (0)
+
+static int host_checks(void) {
+  CHECK(cmr_version() >= 10000);
+  CHECK(strcmp(cmr_status_string(CMR_OK), "CMR_OK") == 0);
+  const int32_t sections[3] = {11, 11, 10};
+  const int32_t bad_sections[3] = {12, 11, 10};
+  /* nothing to do */
+  CHECK(cmr_rotate_qk(NULL, NULL, NULL, 0, 1, 8, 2, 256, 1e7, sections, 64, NULL) == CMR_OK);
+  CHECK(cmr_positions(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL) == CMR_OK);
+  /* rejected before any CUDA call */
+  void* fake = (void*)(uintptr_t)0x10000;
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, 1e7, bad_sections, 64, NULL) == CMR_EINVAL);
+  CHECK(strlen(cmr_last_error_message()) > 0);
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, -1.0, sections, 64, NULL) == CMR_EINVAL);
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 250, 1e7, sections, 64, NULL) == CMR_EINVAL);
+  CHECK(cmr_positions(fake, NULL, 1, 10, 248078, fake, fake, fake, NULL, NULL) == CMR_EINVAL);
+  CHECK(cmr_positions_chunk(fake, fake, 1, 10, 248078, 7, NULL, NULL, NULL, fake, fake, fake,
+                            NULL, NULL) == CMR_EINVAL);
+  CHECK(cmr_copy_rotated_dims(fake, fake, 4, 64, 128, 0, NULL) == CMR_EINVAL);
+  printf("host ok\n");
+  return 0;
+}
+
+/* Just the CUDA runtime calls this program needs, declared here so that the
+ * consumer compiles as plain C with gcc; linked from libcudart. */
+typedef int cuda_err;
+extern cuda_err cudaMalloc(void** p, size_t bytes);
+extern cuda_err cudaFree(void* p);
+extern cuda_err cudaMemcpy(void* dst, const void* src, size_t bytes, int kind);
+extern cuda_err cudaDeviceSynchronize(void);
+
+static int device_run(void) {
+  enum { N = 80, O = 6 };
+  int32_t ids[N], cu[2] = {0, N};
+  for (int p = 0; p < N; ++p) ids[p] = 1000 + p; /* text */
+  ids[O] = 248078;                              /* <image> */
+  for (int k = 0; k < 64; ++k) ids[O + 1 + k] = 248094 + k;
+  ids[O + 65] = 248079;                         /* </image> */
+  ids[O + 66] = 198;                            /* "\n" */
+  int32_t *d_ids, *d_cu, *d_pos, *d_start, *d_amount;
+  CHECK(cudaMalloc((void**)&d_ids, sizeof ids) == 0);
+  CHECK(cudaMalloc((void**)&d_cu, sizeof cu) == 0);
+  CHECK(cudaMalloc((void**)&d_pos, 3 * N * sizeof(int32_t)) == 0);
+  CHECK(cudaMalloc((void**)&d_start, sizeof(int32_t)) == 0);
+  CHECK(cudaMalloc((void**)&d_amount, sizeof(int32_t)) == 0);
+  CHECK(cudaMemcpy(d_ids, ids, sizeof ids, 1) == 0);
+  CHECK(cudaMemcpy(d_cu, cu, sizeof cu, 1) == 0);
+  cmr_status s = cmr_positions(d_ids, d_cu, 1, N, 248078, d_pos, d_start, d_amount, NULL, NULL);
+  if (s != CMR_OK) {
+    fprintf(stderr, "cmr_positions: %s\n", cmr_last_error_message());
+    return 1;
+  }
+  CHECK(cudaDeviceSynchronize() == 0);
+  int32_t pos[3 * N], start, amount;
+  CHECK(cudaMemcpy(pos, d_pos, sizeof pos, 2) == 0);
+  CHECK(cudaMemcpy(&start, d_start, sizeof start, 2) == 0);
+  CHECK(cudaMemcpy(&amount, d_amount, sizeof amount, 2) == 0);
+  for (int p = 0; p < N; ++p) printf("%d %d %d %d\n", p, pos[p], pos[N + p], pos[2 * N + p]);
+  printf("%d %d\n", start, amount);
+  cudaFree(d_ids);
+  cudaFree(d_cu);
+  cudaFree(d_pos);
+  cudaFree(d_start);
+  cudaFree(d_amount);
+  return 0;
+}
+
+int main(int argc, char** argv) {
+  if (argc > 1 && strcmp(argv[1], "device") == 0) return device_run();
+  return host_checks();
+}

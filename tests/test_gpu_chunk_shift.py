@@ -161,3 +161,81 @@ def test_shift_rotate_with_empty_prompts(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(q.view(torch.int16), q2.view(torch.int16))
     assert torch.equal(k.view(torch.int16), k2.view(torch.int16))
+
+
+def test_graph_capture_replays_bit_for_bit(cuda_device):
+    # the library enqueues kernels only (no sync, no allocation), so a CUDA
+    # graph of positions + rotate replays exactly what eager launches do
+    dev = cuda_device
+    wl = inputs.make_config(2, device=dev)
+    ids, cu = t32(wl.ids, dev), t32(wl.cu_seqlens, dev)
+    q0, k0 = wl.q.clone(), wl.k.clone()
+    pos = torch.empty((3, wl.n_tokens), dtype=torch.int32, device=dev)
+    st = torch.empty(wl.num_seqs, dtype=torch.int32, device=dev)
+    am = torch.empty(wl.num_seqs, dtype=torch.int32, device=dev)
+    q, k = q0.clone(), k0.clone()
+    cmr.positions(ids, cu, out=(pos, st, am))
+    cmr.rotate_qk(q, k, pos)
+    torch.cuda.synchronize()
+    eager = (pos.clone(), q.clone(), k.clone())
+    q.copy_(q0)
+    k.copy_(k0)
+    pos.zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        cmr.positions(ids, cu, out=(pos, st, am))
+        cmr.rotate_qk(q, k, pos)
+    q.copy_(q0)
+    k.copy_(k0)
+    pos.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(pos, eager[0])
+    assert torch.equal(q.view(torch.int16), eager[1].view(torch.int16))
+    assert torch.equal(k.view(torch.int16), eager[2].view(torch.int16))
+
+
+@pytest.mark.parametrize("hq,hk,head_dim,rot_dim,sections,L", [
+    (16, 4, 256, 64, (11, 11, 10), 3), (0, 2, 256, 64, (11, 11, 10), 2),
+    (8, 0, 128, 32, (6, 5, 5), 1), (4, 4, 256, 256, (44, 42, 42), 2),
+])
+def test_shift_and_cache_forms_on_other_shapes(cuda_device, hq, hk, head_dim, rot_dim, sections, L):
+    dev = cuda_device
+    rng = np.random.default_rng(hq * 7 + hk)
+    lens = [37, 0, 120, 5, 200]
+    prompts = [inputs.prompt_ids(rng, n, o) for n, o in zip(lens, [3, -1, 0, -1, 50])]
+    ids, cu_np = inputs.pack(prompts)
+    n = ids.size
+    cu = t32(cu_np, dev)
+    pos, s, a = cmr.positions(t32(ids, dev), cu)
+    g = torch.Generator(device=dev).manual_seed(3)
+    mk = lambda h: torch.randn((L, n, h, head_dim), generator=g, device=dev).to(torch.bfloat16) if h else None
+    q, k, v = mk(hq), mk(hk), mk(hk)
+    qa = q.clone() if hq else None
+    ka = k.clone() if hk else None
+    cmr.rotate_qk(qa, ka, pos, 1e7, sections, rot_dim)
+    qb = q.clone() if hq else None
+    kb = k.clone() if hk else None
+    cmr.rotate_qk_shift(qb, kb, s, a, cu_seqlens=cu, theta=1e7, sections=sections, rot_dim=rot_dim)
+    qc = q.clone() if hq else None
+    kc = vc = None
+    if hk:
+        kc = torch.zeros((L, len(lens), hk, 256, head_dim), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+    cmr.rotate_qk_cache(qc, k, v, s, a, kc, vc, cu_seqlens=cu, theta=1e7, sections=sections,
+                        rot_dim=rot_dim)
+    torch.cuda.synchronize()
+    if hq:
+        assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+        assert torch.equal(qa.view(torch.int16), qc.view(torch.int16))
+        p = pos.cpu().numpy()
+        assert_bf16_close(bits(qa), oracle.rotate_bf16(bits(q), p, 1e7, sections, rot_dim), "q")
+    if hk:
+        assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+        for b_ in range(len(lens)):
+            lo, hi = int(cu_np[b_]), int(cu_np[b_ + 1])
+            got_k = kc[:, b_, :, :hi - lo].permute(0, 2, 1, 3)
+            got_v = vc[:, b_, :, :hi - lo].permute(0, 2, 1, 3)
+            assert torch.equal(got_k.contiguous().view(torch.int16), ka[:, lo:hi].view(torch.int16))
+            assert torch.equal(got_v.contiguous().view(torch.int16), v[:, lo:hi].view(torch.int16))
