@@ -58,7 +58,7 @@ def test_rotate_full_compare_small_workloads(cuda_device, cfg):
     check_full(wl.q, wl.k, pos, what=wl.name)
 
 
-@pytest.mark.parametrize("cfg,n_sample", [(3, 3000), (5, 1500)])
+@pytest.mark.parametrize("cfg,n_sample", [(3, 20000), (5, 20000)])
 def test_rotate_full_size_sampled(cuda_device, cfg, n_sample):
     wl = inputs.make_config(cfg, device=cuda_device)
     pos = planes_for(wl, cuda_device)
