@@ -46,6 +46,12 @@ def rotate_bytes(n_tokens, layers, hq, hk, rot_dim):
     return n_tokens * layers * (hq + hk) * rot_dim * 2 * 2 + n_tokens * 12
 
 
+def cache_bytes(n_tokens, layers, hq, hk, rot_dim, head_dim):
+    """Rotate + KV-cache write: Q's rotated dims read and written, K and V rows
+    read and their cache rows written."""
+    return n_tokens * layers * (hq * rot_dim * 2 * 2 + hk * head_dim * 2 * 4)
+
+
 def positions_bytes(n_tokens, num_seqs):
     return n_tokens * 16 + num_seqs * 12
 
@@ -327,21 +333,40 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     tokens_per_step = wl.qk_tokens
     rot_b = rotate_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim)
+    kernel = "rotate_qk_kernel"
+    rope = dict(theta=wl.theta, sections=wl.sections, rot_dim=wl.rot_dim)
 
+    if args.op == "cache":
+        # rotate Q and write rotated K and V rows into [L, B, hk, ctx, D] caches
+        v = inputs.random_qk(tuple(wl.k.shape), wl.seed + 3, dev)
+        ctx = int(wl.cache_len.max()) + 1 if decode else int(np.diff(wl.cu_seqlens).max())
+        k_cache = torch.zeros((L, b, wl.hk, ctx, wl.head_dim), dtype=torch.bfloat16, device=dev)
+        v_cache = torch.zeros_like(k_cache)
+        rot_b = cache_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim, wl.head_dim)
+        kernel = "rotate_qk_cache_kernel"
     if decode:
         # The prompts' (start, amount) come from their prefill, once; a decode
         # step is one launch that derives each new token's planes in the
         # kernel from (cache_len, start, amount) and rotates it.
         cmr.positions(ids, cu, wl.image_token_id, out=(pos, start, amount))
-        plan = [("rotate", lambda: cmr.rotate_qk_shift(wl.q, wl.k, start, amount,
-                                                       pos_offset=cache_len, theta=wl.theta,
-                                                       sections=wl.sections,
-                                                       rot_dim=wl.rot_dim))]
+        if args.op == "cache":
+            plan = [("rotate", lambda: cmr.rotate_qk_cache(
+                wl.q, wl.k, v, start, amount, k_cache, v_cache, pos_offset=cache_len, **rope))]
+        else:
+            plan = [("rotate", lambda: cmr.rotate_qk_shift(wl.q, wl.k, start, amount,
+                                                           pos_offset=cache_len, **rope))]
     else:
         plan = [("positions", lambda: cmr.positions(ids, cu, wl.image_token_id,
-                                                    out=(pos, start, amount))),
-                ("rotate", lambda: cmr.rotate_qk(wl.q, wl.k, pos, wl.theta, wl.sections,
-                                                 wl.rot_dim))]
+                                                    out=(pos, start, amount)))]
+        if args.op == "rotate":
+            plan.append(("rotate", lambda: cmr.rotate_qk(wl.q, wl.k, pos, wl.theta, wl.sections,
+                                                         wl.rot_dim)))
+        elif args.op == "shift":
+            plan.append(("rotate", lambda: cmr.rotate_qk_shift(wl.q, wl.k, start, amount,
+                                                               cu_seqlens=cu, **rope)))
+        else:
+            plan.append(("rotate", lambda: cmr.rotate_qk_cache(
+                wl.q, wl.k, v, start, amount, k_cache, v_cache, cu_seqlens=cu, **rope)))
     calls = dict(plan)
     if args.launch == "graph":
         # one CUDA graph per call, each holding its single kernel launch
@@ -395,13 +420,17 @@ def run_ours(args):
     launches = args.steps * len(plan)
 
     # end to end through the public API from pinned host memory
-    e2e = run_e2e(args, wl, dev, stream, dist, tokens_all)
+    if args.op == "rotate":
+        e2e = run_e2e(args, wl, dev, stream, dist, tokens_all)
+    else:
+        e2e = {"skipped": f"--op {args.op} times the device step only; the end-to-end path "
+                          "is measured with --op rotate"}
 
     if rank == 0:
         peak, peak_src = measured_peak()
         rot_avg_s = statistics.mean(rot_ms) / 1e3
         achieved = rot_b / rot_avg_s / 1e9
-        traffic = recorded_traffic(wl.name)
+        traffic = recorded_traffic(wl.name) if args.op == "rotate" else None
         value = tokens_all * args.steps / (ms_max / 1e3)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -414,7 +443,7 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,1) bf16 Q/K, uniform text ids, one 448x448 frame "
                     "per prompt)",
             "config": {"workload": workload_label(wl), "global_batch": tokens_all,
-                       "launch": args.launch,
+                       "launch": args.launch, "op": args.op,
                        "seq_len": n // max(b, 1),
                        "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'whole prompts split over ranks'}, no data-path collective)",
                        "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
@@ -423,7 +452,7 @@ def run_ours(args):
             "token_layers_per_s": value * L,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "rotate_qk_kernel",
+                         "kernel": kernel,
                          "algorithmic_bytes_per_launch": rot_b,
                          "avg_launch_ms": rot_avg_s * 1e3,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
@@ -528,6 +557,9 @@ def main():
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: a full batch per GPU (default); strong: one batch split by "
                          "whole prompts")
+    ap.add_argument("--op", choices=["rotate", "shift", "cache"], default="rotate",
+                    help="rotate: planes from pos (default); shift: planes derived in the "
+                         "rotate kernel; cache: rotate + KV-cache write")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="graph: replay a captured CUDA graph per call (default); eager: "
                          "launch through the Python binding every step")
