@@ -36,7 +36,10 @@ METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
-                  "vlm_decoder_positional_b200/csrc/cmr_internal.cuh"]
+                  "vlm_decoder_positional_b200/csrc/rotate_common.cuh",
+                  "vlm_decoder_positional_b200/csrc/canvas.cuh",
+                  "vlm_decoder_positional_b200/csrc/cmr_internal.cuh",
+                  "include/cmr.h"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rotate_qk_traffic.txt")
 
 # Algorithmic bytes: rotate reads and writes the rot_dim dims of every Q and K
