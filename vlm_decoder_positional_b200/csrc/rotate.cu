@@ -23,8 +23,9 @@
 // is 8 tokens x 64 contiguous bytes (whole 32-B sectors), and the x / partner
 // loads of one head row together cover its 128-B line.  kBatch head rows are
 // loaded (two 16-byte loads each, evict-first) before any is rotated and
-// stored back (two 16-byte stores each).  Tiles of many rows get one CTA
-// each (a one-shot grid); tiles of few rows are walked by a persistent grid.
+// stored back (two 16-byte stores each); kBatch is 4, or 5 where that saves a
+// load round.  Tiles of many rows get one CTA each (a one-shot grid); tiles
+// of few rows are walked by a persistent grid (choose_plan has the numbers).
 // When a batch has too few tokens to fill the GPU (decode), each token's
 // (layer, head) rows are split into groups handled by different threads,
 // each computing the same 8 cos/sin.
@@ -38,12 +39,23 @@ namespace {
 using namespace rot;
 
 constexpr int kThreads = 128;
-constexpr int kMinBlocksPerSm = 4;
-constexpr int kBatch = 4;  // head rows in flight per thread
 constexpr int kOneShotRows = 16;  // rows per item from which a CTA serves one tile
 
-template <bool kFromShift>
-__global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
+// kBatch head rows are in flight per thread; the launch bounds keep the
+// batch's registers within the occupancy each variant was tuned for.
+template <int kBatch>
+struct BatchShape;
+template <>
+struct BatchShape<4> {
+  static constexpr int kMinBlocksPerSm = 4;
+};
+template <>
+struct BatchShape<5> {
+  static constexpr int kMinBlocksPerSm = 3;
+};
+
+template <bool kFromShift, int kBatch>
+__global__ void __launch_bounds__(kThreads, BatchShape<kBatch>::kMinBlocksPerSm)
     rotate_qk_kernel(const RotateArgs args, const FreqTable table) {
   __shared__ double s_inv[kMaxFreqs];
   __shared__ int32_t s_plane[kMaxFreqs];
@@ -141,36 +153,66 @@ __global__ void __launch_bounds__(kThreads, kMinBlocksPerSm)
   }
 }
 
+// The kernel variants: plane source x rows in flight per thread (4 or 5).
+using KernelFn = void (*)(RotateArgs, FreqTable);
+KernelFn variant(bool from_shift, int batch_index) {
+  static const KernelFn table[2][2] = {
+      {rotate_qk_kernel<false, 4>, rotate_qk_kernel<false, 5>},
+      {rotate_qk_kernel<true, 4>, rotate_qk_kernel<true, 5>}};
+  return table[from_shift ? 1 : 0][batch_index];
+}
+
 struct OccupancyCache {
   std::mutex mu;
   int device = -1;
-  int ctas[2] = {0, 0};
+  int ctas[2][2] = {};
 };
 OccupancyCache g_occ[64];
 
 // CTAs of each variant resident on the whole device at full occupancy
 // (cached per device).
-cudaError_t resident_ctas(bool from_shift, int* total) {
+cudaError_t resident_ctas(bool from_shift, int batch_index, int* total) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   OccupancyCache& c = g_occ[dev & 63];
   std::lock_guard<std::mutex> lock(c.mu);
   if (c.device != dev) {
-    int sms = 0, per_sm[2] = {0, 0};
+    int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[0], rotate_qk_kernel<false>,
-                                                      kThreads, 0);
-    if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[1], rotate_qk_kernel<true>,
-                                                      kThreads, 0);
-    if (e != cudaSuccess) return e;
+    for (int f = 0; f < 2; ++f)
+      for (int bi = 0; bi < 2; ++bi) {
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, variant(f == 1, bi), kThreads, 0);
+        if (e != cudaSuccess) return e;
+        c.ctas[f][bi] = sms * (per_sm > 0 ? per_sm : 1);
+      }
     c.device = dev;
-    for (int i = 0; i < 2; ++i) c.ctas[i] = sms * (per_sm[i] > 0 ? per_sm[i] : 1);
   }
-  *total = c.ctas[from_shift ? 1 : 0];
+  *total = c.ctas[from_shift ? 1 : 0][batch_index];
   return cudaSuccess;
+}
+
+// Rows in flight per thread and grid shape for a given number of rows per
+// work item.
+struct Plan {
+  int batch_index;  // 0: 4 rows in flight per thread, 1: 5 rows
+  bool one_shot;    // one CTA per tile, else a persistent grid of resident CTAs
+};
+// Measured on B200 (64 x 4096 tokens, graph replay):
+//  - from 16 rows per item (2+ layers of 8 + 2 heads) one CTA per tile beats a
+//    persistent grid, 6.02-6.12 vs 5.85-5.92 TB/s: the scheduler hands CTAs out
+//    as earlier ones finish and the addresses in flight stay in one window;
+//  - where 5 rows per batch saves a load round (5, 9 or 10 rows: one layer of
+//    8 + 2 heads takes 2 rounds instead of 3), 5 rows with one CTA per tile win,
+//    5.82 vs 5.65 TB/s (4 rows, persistent) and 5.40 (4 rows, one-shot);
+//  - otherwise a persistent grid, whose one-item-ahead plane prefetch hides the
+//    planes' latency.
+Plan choose_plan(int rows_per_item) {
+  const bool fewer_rounds_with_5 = (rows_per_item + 4) / 5 < (rows_per_item + 3) / 4;
+  if (rows_per_item <= 10 && fewer_rounds_with_5) return {1, true};
+  return {0, rows_per_item >= kOneShotRows};
 }
 
 }  // namespace
@@ -178,32 +220,28 @@ cudaError_t resident_ctas(bool from_shift, int* total) {
 cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream) {
   RotateArgs a = in;
   const bool from_shift = a.pos == nullptr;
-  int max_ctas = 0;
-  cudaError_t e = resident_ctas(from_shift, &max_ctas);
-  if (e != cudaSuccess) return e;
   const int64_t items_per_cta = kThreads / a.units_per_head;
   // Split each token's (layer, head) rows into groups only when there are too
-  // few tokens to fill one wave of resident CTAs.
+  // few tokens to fill one wave of resident CTAs (sized with the default
+  // variant).
+  int wave_ctas = 0;
+  cudaError_t e = resident_ctas(from_shift, 0, &wave_ctas);
+  if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(a.hq + a.hk) * a.num_layers;
-  const int64_t wave_items = static_cast<int64_t>(max_ctas) * items_per_cta;
+  const int64_t wave_items = static_cast<int64_t>(wave_ctas) * items_per_cta;
   int64_t groups = (wave_items + a.n_tokens - 1) / a.n_tokens;
   groups = groups < 1 ? 1 : (groups > rows ? rows : groups);
   a.jobs_per_group = static_cast<int32_t>((rows + groups - 1) / groups);
   a.job_groups = static_cast<int32_t>((rows + a.jobs_per_group - 1) / a.jobs_per_group);
+  const Plan plan = choose_plan(a.jobs_per_group);
+  int max_ctas = 0;
+  e = resident_ctas(from_shift, plan.batch_index, &max_ctas);
+  if (e != cudaSuccess) return e;
   const int64_t items = a.n_tokens * a.job_groups;
   const int64_t needed = (items + items_per_cta - 1) / items_per_cta;
-  // Grid shape (measured on B200, 64 x 4096 tokens): with many rows per item
-  // one CTA per tile (the scheduler hands CTAs out as others finish, keeping
-  // the addresses in flight in one moving window) beats a persistent grid,
-  // 6.0-6.1 vs 5.85-5.9 TB/s from 2 layers on; with few rows per item the
-  // persistent grid's one-item-ahead plane prefetch wins (5.64 vs 5.40 TB/s
-  // at 1 layer).
-  const int64_t ctas = (a.jobs_per_group >= kOneShotRows || needed <= max_ctas)
-                           ? needed : max_ctas;
-  if (from_shift)
-    rotate_qk_kernel<true><<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
-  else
-    rotate_qk_kernel<false><<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(a, table);
+  const int64_t ctas = (plan.one_shot || needed <= max_ctas) ? needed : max_ctas;
+  variant(from_shift, plan.batch_index)<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(
+      a, table);
   return cudaGetLastError();
 }
 
