@@ -12,6 +12,15 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+@pytest.fixture(scope="session", autouse=True)
+def _built_libraries():
+    """Build libcmr.so (nvcc) and the oracle (gcc) when missing or stale."""
+    from oracle import build as oracle_build
+    from vlm_decoder_positional_b200 import build as libbuild
+    libbuild.build()
+    oracle_build.build()
+
+
 @pytest.fixture(scope="session")
 def cuda_device():
     import torch
