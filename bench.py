@@ -18,6 +18,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -75,11 +76,36 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def rotate_source_hash():
+_C_TOKENS = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\\n])*"|\'(?:\\.|[^\'\\\n])*\'|\s+|[^\s"\'/]+|/',
+                       re.S)
+
+
+def code_tokens(text):
+    """The source with comments dropped and every run of whitespace folded to one
+    space (string and character literals kept as written), so that a comment
+    edit does not count as a change of the kernel."""
+    out = []
+    for m in _C_TOKENS.finditer(text):
+        tok = m.group(0)
+        if tok.startswith("//") or tok.startswith("/*") or tok.isspace():
+            if out and out[-1] != " ":
+                out.append(" ")
+        else:
+            out.append(tok)
+    return "".join(out).strip()
+
+
+def rotate_source_hash(read=None):
+    """SHA-256 of the code (comments and layout aside) of every source the
+    rotate kernel compiles; `read(rel)` returns a file's text (default: this
+    checkout)."""
+    if read is None:
+        def read(rel):
+            with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+                return f.read()
     h = hashlib.sha256()
     for rel in ROTATE_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        h.update(rel.encode() + b"\0" + code_tokens(read(rel)).encode() + b"\0")
     return h.hexdigest()
 
 

@@ -123,6 +123,8 @@ CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
  *   out_start, out_amount device int32 [num_seqs]: the state after the chunk.
  *                   Must not overlap in_start / in_amount (use two buffers and
  *                   swap them between chunks).
+ * Absolute indices (pos_offset[b] plus the chunk's length) must stay below
+ * 2^30 - 67: a start of 2^30 or more reads as "no frame seen".
  * Errors: as cmr_positions, plus CMR_EINVAL for an unknown rule or
  * overlapping incoming and outgoing state. */
 CMR_API cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens,
@@ -230,7 +232,9 @@ CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqle
  *   cu_seqlens, num_seqs, pos_offset, start, amount   as in cmr_rotate_qk_shift
  *   the rest           as in cmr_rotate_qk
  * All of q, k, v, k_cache, v_cache 16-byte aligned; the caches must not
- * overlap q, k or v.
+ * overlap q, k or v.  Two tokens that land on the same (slot, position) --
+ * sequences sharing a slot, or repeated indices -- race; give each sequence
+ * its own slot.
  * Errors: as cmr_rotate_qk_shift, plus CMR_EINVAL for missing or misaligned
  * v / caches or non-positive cache sizes. */
 CMR_API cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v,

@@ -24,6 +24,22 @@ def test_traffic_record_is_tied_to_the_kernel_source_and_workload():
     assert bench.recorded_traffic("some_other_workload") is None
 
 
+def test_source_hash_ignores_comments_but_not_code():
+    src = {rel: open(os.path.join(bench.ROOT, rel)).read() for rel in bench.ROTATE_SOURCES}
+    base = bench.rotate_source_hash(src.__getitem__)
+    assert base == bench.rotate_source_hash()
+    rel = "vlm_decoder_positional_b200/csrc/rotate.cu"
+    commented = dict(src)
+    commented[rel] = "// a new remark\n" + src[rel].replace("\n", "\n  /* note */\n", 3)
+    assert bench.rotate_source_hash(commented.__getitem__) == base
+    changed = dict(src)
+    changed[rel] = src[rel].replace("kOneShotRows = 16", "kOneShotRows = 17")
+    assert changed[rel] != src[rel]
+    assert bench.rotate_source_hash(changed.__getitem__) != base
+    # a "//" inside a string literal is code, not a comment
+    assert bench.code_tokens('f("a//b"); // c') == 'f("a//b");'
+
+
 def test_oracle_sample_step_threads_agree():
     wl = inputs.make_config(2)
     wl_cpu = bench.cpu_sample_inputs(wl, 600)
