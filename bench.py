@@ -37,6 +37,8 @@ METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
+                  "vlm_decoder_positional_b200/csrc/rotate_staged.cu",
+                  "vlm_decoder_positional_b200/csrc/tma.cuh",
                   "vlm_decoder_positional_b200/csrc/rotate_common.cuh",
                   "vlm_decoder_positional_b200/csrc/canvas.cuh",
                   "vlm_decoder_positional_b200/csrc/cmr_internal.cuh",
@@ -109,9 +111,9 @@ def rotate_source_hash(read=None):
     return h.hexdigest()
 
 
-def recorded_traffic(workload_name):
+def recorded_traffic(workload_name, kernel=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    this exact kernel source and workload; otherwise None."""
+    this exact kernel source, workload and kernel; otherwise None."""
     try:
         rec = {}
         with open(TRAFFIC_FILE) as f:
@@ -122,6 +124,8 @@ def recorded_traffic(workload_name):
         if rec.get("kernel_source_sha256") != rotate_source_hash():
             return None
         if rec.get("workload") != workload_name:
+            return None
+        if kernel is not None and rec.get("kernel") != kernel:
             return None
         return int(rec["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -371,7 +375,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     tokens_per_step = wl.qk_tokens
     rot_b = rotate_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim)
-    kernel = "rotate_qk_kernel"
+    # the kernel the library picks for this shape (staged or register-resident)
+    kernel = cmr.rotate_qk_kernel(wl.qk_tokens, L, wl.hq, wl.hk, wl.head_dim, wl.rot_dim)
     rope = dict(theta=wl.theta, sections=wl.sections, rot_dim=wl.rot_dim)
 
     if args.op == "cache":
@@ -468,7 +473,7 @@ def run_ours(args):
         peak, peak_src = measured_peak()
         rot_avg_s = statistics.mean(rot_ms) / 1e3
         achieved = rot_b / rot_avg_s / 1e9
-        traffic = recorded_traffic(wl.name) if args.op == "rotate" else None
+        traffic = recorded_traffic(wl.name, kernel) if args.op == "rotate" else None
         value = tokens_all * args.steps / (ms_max / 1e3)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:

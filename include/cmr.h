@@ -22,8 +22,9 @@
  *     non-CMR_OK return nothing was enqueued, except CMR_ECUDA from a launch,
  *     which means the launch itself failed.  cmr_last_error_message() then
  *     gives a one-line reason (per calling thread).
- *   - Kernels never trap.  Malformed device-side data (cu_seqlens) is reported
- *     through an optional device status word.
+ *   - Kernels never trap.  Malformed device-side data (cu_seqlens, cache
+ *     indices) and a staged copy that never arrived are reported through an
+ *     optional device status word; every wait inside a kernel is bounded.
  */
 #ifndef CMR_H_
 #define CMR_H_
@@ -53,6 +54,8 @@ typedef enum cmr_status {
 /* Bits a kernel ORs into the optional device status word. */
 #define CMR_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens not 0 .. n_tokens, non-decreasing */
 #define CMR_DEVICE_CACHE_RANGE 2    /* a token's cache index or slot outside the cache */
+#define CMR_DEVICE_WAIT_TIMEOUT 4   /* a staged kernel waited over 1 s for a copy and gave
+                                       up; rows of the tiles involved may be unrotated */
 
 /* Position rules for cmr_positions_chunk. */
 #define CMR_RULE_CANVAS 0    /* this model's canvas rule: start = O + 67, amount 58 */
@@ -165,7 +168,8 @@ CMR_API cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* s
  *   x_{j+F} <- x_{j+F} cos a + x_j sin a
  * Dims rot_dim .. head_dim-1 are not read or written.  The angle is formed and
  * reduced modulo 2*pi in fp64, cos/sin and the rotation run in fp32, and the
- * result is rounded to bf16 (nearest-even).
+ * result is rounded to bf16 (nearest-even).  Large batches with rot_dim 64 run
+ * a TMA-staged kernel; the result is the same bit for bit either way.
  *
  *   q      device bf16 [num_layers, n_tokens, hq, head_dim], 16-byte aligned
  *   k      device bf16 [num_layers, n_tokens, hk, head_dim], 16-byte aligned
@@ -178,13 +182,15 @@ CMR_API cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* s
  *   sections  host int32 [3] = {T, H, W} frequency counts, summing to
  *          rot_dim / 2, each realisable by the interleave above
  *   rot_dim   multiple of 16, 16 .. min(head_dim, 256)  (64 for this model)
+ *   device_status  optional device int32 [1] (may be NULL): receives
+ *          CMR_DEVICE_WAIT_TIMEOUT if a staged copy timed out.  Never cleared.
  * Errors: CMR_EINVAL for any violation above; CMR_EUNSUPPORTED when
  * (hq + hk) * num_layers > INT32_MAX. */
 CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
                          int32_t num_layers, int32_t hq, int32_t hk,
                          int32_t head_dim, double theta,
                          const int32_t sections[3], int32_t rot_dim,
-                         cmr_stream_t stream);
+                         int32_t* device_status, cmr_stream_t stream);
 
 /* cmr_rotate_qk with the planes derived inside the kernel instead of read
  * from pos [3, n_tokens]: token t of prompt b (cu[b] <= t < cu[b+1]) sits at
@@ -194,8 +200,8 @@ CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n
  * (cu_seqlens = NULL: token b is sequence b, p = pos_offset[b]) or a prefill
  * chunk whose state is known, and the 24 B/token pos round trip disappears.
  *
- *   q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections, rot_dim
- *                 as in cmr_rotate_qk
+ *   q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections, rot_dim,
+ *   device_status as in cmr_rotate_qk
  *   cu_seqlens    device int32 [num_seqs + 1] as in cmr_positions (it must be
  *                 well formed: it is not checked on the device), or NULL when
  *                 num_seqs == n_tokens and each sequence holds one token
@@ -209,7 +215,18 @@ CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqle
                                        int64_t n_tokens, int32_t num_layers, int32_t hq,
                                        int32_t hk, int32_t head_dim, double theta,
                                        const int32_t sections[3], int32_t rot_dim,
-                                       cmr_stream_t stream);
+                                       int32_t* device_status, cmr_stream_t stream);
+
+/* Name of the kernel that cmr_rotate_qk / cmr_rotate_qk_shift launch for these
+ * shapes: "rotate_qk_staged_kernel" (TMA-staged, rot_dim 64, large batches) or
+ * "rotate_qk_kernel" (register-resident rows, every other case).  The staged
+ * kernel also needs the driver to encode tensor maps for the buffers (any
+ * driver for sm_100a does, for contiguous Q/K of under 1 TB per layer);
+ * otherwise the call takes rotate_qk_kernel.
+ * Returns NULL when the shapes are invalid or there is nothing to launch.
+ * Static strings; no CUDA call is made. */
+CMR_API const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, int32_t hq,
+                                         int32_t hk, int32_t head_dim, int32_t rot_dim);
 
 /* Rotate Q in place and write each token's rotated K row and its V row into
  * a KV cache, in one pass: the step after the rotation in the full-attention

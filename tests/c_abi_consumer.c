@@ -20,19 +20,19 @@
   } while (0)
 
 static int host_checks(void) {
-  CHECK(cmr_version() >= 10000);
+  CHECK(cmr_version() >= 20000);
   CHECK(strcmp(cmr_status_string(CMR_OK), "CMR_OK") == 0);
   const int32_t sections[3] = {11, 11, 10};
   const int32_t bad_sections[3] = {12, 11, 10};
   /* nothing to do */
-  CHECK(cmr_rotate_qk(NULL, NULL, NULL, 0, 1, 8, 2, 256, 1e7, sections, 64, NULL) == CMR_OK);
+  CHECK(cmr_rotate_qk(NULL, NULL, NULL, 0, 1, 8, 2, 256, 1e7, sections, 64, NULL, NULL) == CMR_OK);
   CHECK(cmr_positions(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL) == CMR_OK);
   /* rejected before any CUDA call */
   void* fake = (void*)(uintptr_t)0x10000;
-  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, 1e7, bad_sections, 64, NULL) == CMR_EINVAL);
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, 1e7, bad_sections, 64, NULL, NULL) == CMR_EINVAL);
   CHECK(strlen(cmr_last_error_message()) > 0);
-  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, -1.0, sections, 64, NULL) == CMR_EINVAL);
-  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 250, 1e7, sections, 64, NULL) == CMR_EINVAL);
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 256, -1.0, sections, 64, NULL, NULL) == CMR_EINVAL);
+  CHECK(cmr_rotate_qk(fake, fake, fake, 10, 1, 8, 2, 250, 1e7, sections, 64, NULL, NULL) == CMR_EINVAL);
   CHECK(cmr_positions(fake, NULL, 1, 10, 248078, fake, fake, fake, NULL, NULL) == CMR_EINVAL);
   CHECK(cmr_positions_chunk(fake, fake, 1, 10, 248078, 7, NULL, NULL, NULL, fake, fake, fake,
                             NULL, NULL) == CMR_EINVAL);

@@ -28,7 +28,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
-                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache",
+                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache", "cmr_rotate_qk_kernel",
                           "cmr_copy_rotated_dims", "cmr_status_string",
                           "cmr_last_error_message", "cmr_version"}
     assert set(names) == set(cmr.SIGNATURES)
@@ -49,7 +49,7 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 10300
+    assert lib.cmr_version() == 20000
 
 
 SEC = (ctypes.c_int32 * 3)(11, 11, 10)
@@ -69,19 +69,19 @@ def test_rotate_rejects_bad_arguments_on_the_host(lib, kw):
     a.update(kw)
     sec = None if a["sections"] is None else (ctypes.c_int32 * 3)(*a["sections"])
     st = lib.cmr_rotate_qk(a["q"], a["k"], a["pos"], a["n_tokens"], a["num_layers"], a["hq"],
-                           a["hk"], a["head_dim"], a["theta"], sec, a["rot_dim"], None)
+                           a["hk"], a["head_dim"], a["theta"], sec, a["rot_dim"], None, None)
     assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
     assert lib.cmr_last_error_message()
 
 
 def test_rotate_too_many_head_rows_is_unsupported(lib):
-    st = lib.cmr_rotate_qk(FAKE, FAKE, FAKE, 10, 80000, 30000, 2, 256, 1e7, SEC, 64, None)
+    st = lib.cmr_rotate_qk(FAKE, FAKE, FAKE, 10, 80000, 30000, 2, 256, 1e7, SEC, 64, None, None)
     assert st == cmr.CMR_EUNSUPPORTED
 
 
 def test_rotate_empty_work_is_a_no_op(lib):
-    assert lib.cmr_rotate_qk(None, None, None, 0, 1, 8, 2, 256, 1e7, SEC, 64, None) == 0
-    assert lib.cmr_rotate_qk(None, None, None, 10, 0, 8, 2, 256, 1e7, SEC, 64, None) == 0
+    assert lib.cmr_rotate_qk(None, None, None, 0, 1, 8, 2, 256, 1e7, SEC, 64, None, None) == 0
+    assert lib.cmr_rotate_qk(None, None, None, 10, 0, 8, 2, 256, 1e7, SEC, 64, None, None) == 0
 
 
 @pytest.mark.parametrize("args", [
@@ -124,7 +124,7 @@ def test_rotate_shift_rejects_bad_arguments_on_the_host(lib, kw):
              rot_dim=64)
     a.update(kw)
     st = lib.cmr_rotate_qk_shift(a["q"], a["k"], a["cu"], a["num_seqs"], a["off"], a["start"],
-                                 a["amount"], a["n"], 1, 8, 2, 256, 1e7, SEC, a["rot_dim"], None)
+                                 a["amount"], a["n"], 1, 8, 2, 256, 1e7, SEC, a["rot_dim"], None, None)
     assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
 
 
@@ -151,3 +151,24 @@ def test_copy_rotated_dims_rejects_bad_arguments(lib, args):
 
 def test_copy_rotated_dims_of_nothing_is_a_no_op(lib):
     assert lib.cmr_copy_rotated_dims(None, None, 0, 256, 64, 0, None) == cmr.CMR_OK
+
+
+def test_kernel_query_names_the_path_each_shape_takes(lib):
+    def name(*a):
+        r = lib.cmr_rotate_qk_kernel(*a)
+        return None if r is None else r.decode()
+    staged, regs = "rotate_qk_staged_kernel", "rotate_qk_kernel"
+    assert name(262144, 6, 8, 2, 256, 64) == staged      # the 6-layer prefill batch
+    assert name(262144, 1, 8, 2, 256, 64) == staged
+    assert name(8192, 6, 8, 2, 256, 64) == staged        # 1024 tiles of 8 tokens
+    assert name(8185, 6, 8, 2, 256, 64) == staged        # 1024 tiles, the last of one token
+    assert name(8184, 6, 8, 2, 256, 64) == regs          # 1023 tiles
+    assert name(1024, 6, 8, 2, 256, 64) == regs          # a decode step
+    assert name(262144, 6, 8, 2, 256, 128) == regs       # rot_dim other than 64
+    assert name(262144, 2, 64, 64, 256, 64) == regs      # a stage of 128 head rows is too big
+    assert name(262144, 2, 16, 4, 256, 64) == staged
+    assert name(262144, 2, 0, 3, 128, 64) == staged
+    for bad in [(0, 6, 8, 2, 256, 64), (10, 0, 8, 2, 256, 64), (10, 1, 0, 0, 256, 64),
+                (10, 1, 8, 2, 250, 64), (10, 1, 8, 2, 256, 24), (10, 1, 8, 2, 32, 64),
+                (10, 80000, 30000, 2, 256, 64), (-1, 1, 8, 2, 256, 64)]:
+        assert name(*bad) is None, bad

@@ -19,9 +19,10 @@ def test_algorithmic_bytes_match_the_hand_count():
 
 
 def test_traffic_record_is_tied_to_the_kernel_source_and_workload():
-    t = bench.recorded_traffic("c5_6layers_32x8192")
+    t = bench.recorded_traffic("c5_6layers_32x8192", "rotate_qk_staged_kernel")
     assert t is None or 3.5e9 < t < 4.5e9
     assert bench.recorded_traffic("some_other_workload") is None
+    assert bench.recorded_traffic("c5_6layers_32x8192", "rotate_qk_kernel") is None
 
 
 def test_source_hash_ignores_comments_but_not_code():

@@ -170,9 +170,86 @@ def test_misaligned_and_host_pointers_are_rejected(cuda_device):
     sec = cmr.ctypes.c_int32 * 3
     L = cmr.lib()
     rc = L.cmr_rotate_qk(q.data_ptr() + 2, k.data_ptr(), pos.data_ptr(), 4, 1, 8, 2, 256, 1e7,
-                         sec(11, 11, 10), 64, None)
+                         sec(11, 11, 10), 64, None, None)
     assert rc == cmr.CMR_EINVAL
     host = np.zeros(4 * 8 * 256, np.uint16)
     rc = L.cmr_rotate_qk(host.ctypes.data, k.data_ptr(), pos.data_ptr(), 4, 1, 8, 2, 256, 1e7,
-                         sec(11, 11, 10), 64, None)
+                         sec(11, 11, 10), 64, None, None)
     assert rc == cmr.CMR_EINVAL
+
+
+# ---- the TMA-staged kernel (rot_dim 64, from 1024 tiles of 8 tokens) ----
+
+STAGED_MIN_TOKENS = 1024 * 8
+
+
+@pytest.mark.parametrize("n", [STAGED_MIN_TOKENS, STAGED_MIN_TOKENS + 1, STAGED_MIN_TOKENS + 7,
+                               10001])
+@pytest.mark.parametrize("layers", [1, 3, 4, 5, 9])
+def test_rotate_staged_ragged_tiles_and_ring_wrap(cuda_device, n, layers):
+    # tiles of 8 tokens with a ragged last tile; 4, 5 and 9 layers wrap the
+    # 3-stage ring
+    assert cmr.rotate_qk_kernel(n, layers, 8, 2) == "rotate_qk_staged_kernel"
+    g = torch.Generator(device=cuda_device).manual_seed(n + 100 * layers)
+    q = torch.randn((layers, n, 8, 256), generator=g, device=cuda_device).to(torch.bfloat16)
+    k = torch.randn((layers, n, 2, 256), generator=g, device=cuda_device).to(torch.bfloat16)
+    pos = torch.randint(-70, 400000, (3, n), generator=g, device=cuda_device, dtype=torch.int32)
+    check_full(q, k, pos, what=f"staged n={n} L={layers}")
+
+
+@pytest.mark.parametrize("hq,hk,head_dim", [(16, 4, 256), (1, 0, 256), (0, 3, 128), (8, 2, 64),
+                                            (8, 2, 72), (3, 1, 256)])
+def test_rotate_staged_other_heads_and_head_dims(cuda_device, hq, hk, head_dim):
+    g = torch.Generator(device=cuda_device).manual_seed(hq * 1000 + hk * 10 + head_dim)
+    n, L = 9001, 2
+    assert cmr.rotate_qk_kernel(n, L, hq, hk, head_dim) == "rotate_qk_staged_kernel"
+    q = (torch.randn((L, n, hq, head_dim), generator=g, device=cuda_device).to(torch.bfloat16)
+         if hq else None)
+    k = (torch.randn((L, n, hk, head_dim), generator=g, device=cuda_device).to(torch.bfloat16)
+         if hk else None)
+    pos = torch.randint(0, 30000, (3, n), generator=g, device=cuda_device, dtype=torch.int32)
+    check_full(q, k, pos, what=f"staged {hq},{hk},{head_dim}")
+
+
+def test_staged_and_register_kernels_agree_bit_for_bit(cuda_device):
+    # the whole batch takes the staged kernel; the same rows rotated 512
+    # tokens at a time take the register kernel: identical bits
+    n, L = 20000, 6
+    g = torch.Generator(device=cuda_device).manual_seed(11)
+    q = inputs.random_qk((L, n, 8, 256), 5, cuda_device)
+    k = inputs.random_qk((L, n, 2, 256), 6, cuda_device)
+    pos = torch.randint(-(2 ** 20), 2 ** 20, (3, n), generator=g, device=cuda_device,
+                        dtype=torch.int32)
+    q2, k2 = q.clone(), k.clone()
+    assert cmr.rotate_qk_kernel(n, L, 8, 2) == "rotate_qk_staged_kernel"
+    assert cmr.rotate_qk_kernel(512, L, 8, 2) == "rotate_qk_kernel"
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    cmr.rotate_qk(q, k, pos, device_status=status)
+    for a in range(0, n, 512):
+        b = min(n, a + 512)
+        qc, kc = q2[:, a:b].contiguous(), k2[:, a:b].contiguous()
+        cmr.rotate_qk(qc, kc, pos[:, a:b].contiguous(), device_status=status)
+        q2[:, a:b], k2[:, a:b] = qc, kc
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(q.view(torch.int16), q2.view(torch.int16))
+    assert torch.equal(k.view(torch.int16), k2.view(torch.int16))
+
+
+def test_staged_shift_form_matches_pos_form(cuda_device):
+    # planes derived in the staged kernel from (start, amount) equal the pos
+    # form's result, bit for bit, on a prefill batch large enough to stage
+    wl = inputs.make_config(3, device=cuda_device)
+    ids = torch.from_numpy(wl.ids).to(cuda_device)
+    cu = torch.from_numpy(wl.cu_seqlens).to(cuda_device)
+    pos, start, amount = cmr.positions(ids, cu, wl.image_token_id)
+    assert cmr.rotate_qk_kernel(wl.n_tokens, wl.num_layers, wl.hq, wl.hk) == \
+        "rotate_qk_staged_kernel"
+    q2, k2 = wl.q.clone(), wl.k.clone()
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    cmr.rotate_qk(wl.q, wl.k, pos, device_status=status)
+    cmr.rotate_qk_shift(q2, k2, start, amount, cu_seqlens=cu, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(wl.q.view(torch.int16), q2.view(torch.int16))
+    assert torch.equal(wl.k.view(torch.int16), k2.view(torch.int16))

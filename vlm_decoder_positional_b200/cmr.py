@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libcmr.so")
 CMR_OK, CMR_EINVAL, CMR_ECUDA, CMR_EUNSUPPORTED = 0, 1, 2, 3
 CMR_DEVICE_BAD_CU_SEQLENS = 1
 CMR_DEVICE_CACHE_RANGE = 2
+CMR_DEVICE_WAIT_TIMEOUT = 4
 RULES = {"canvas": 0, "qwen_vl": 1, "planes_1d": 2}
 TEXT_ONLY_START = 1 << 30
 
@@ -37,7 +38,7 @@ SIGNATURES = {
                                            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_int32, ctypes.c_double,
                                            ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
-                                           ctypes.c_void_p]),
+                                           _i32p, ctypes.c_void_p]),
     "cmr_rotate_qk_cache": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                            _i32p, ctypes.c_int32, _i32p, _i32p, _i32p,
                                            ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
@@ -49,7 +50,9 @@ SIGNATURES = {
                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.c_double,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
-                                     ctypes.c_void_p]),
+                                     _i32p, ctypes.c_void_p]),
+    "cmr_rotate_qk_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "cmr_copy_rotated_dims": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_void_p]),
@@ -110,6 +113,13 @@ def _want(t: torch.Tensor, name: str, dtype: torch.dtype, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _status_ptr(device_status: Optional[torch.Tensor], dev) -> Optional[int]:
+    if device_status is None:
+        return None
+    _want(device_status, "device_status", torch.int32, dev)
+    return device_status.data_ptr()
 
 
 def positions(ids: torch.Tensor, cu_seqlens: torch.Tensor, image_token_id: int = IMAGE_TOKEN_ID,
@@ -252,10 +262,12 @@ def rotate_qk_shift(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                     cu_seqlens: Optional[torch.Tensor] = None,
                     pos_offset: Optional[torch.Tensor] = None, theta: float = 1e7,
                     sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
-                    stream: Optional[torch.cuda.Stream] = None):
+                    stream: Optional[torch.cuda.Stream] = None,
+                    device_status: Optional[torch.Tensor] = None):
     """cmr_rotate_qk_shift, in place: the planes of token t of prompt b are the
     canvas rows at pos_offset[b] + t - cu[b] under (start[b], amount[b]);
-    cu_seqlens=None means one token per sequence (a decode step)."""
+    cu_seqlens=None means one token per sequence (a decode step).
+    device_status: optional int32 [1] on the device (CMR_DEVICE_* bits)."""
     _want(start, "start", torch.int32)
     dev = start.device
     _want(amount, "amount", torch.int32, dev)
@@ -276,13 +288,15 @@ def rotate_qk_shift(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
         if pos_offset.numel() != b:
             raise ValueError("pos_offset needs num_seqs entries")
         off_ptr = pos_offset.data_ptr()
+    st_ptr = _status_ptr(device_status, dev)
     sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
     with torch.cuda.device(dev):
         _check(lib().cmr_rotate_qk_shift(
             q.data_ptr() if q is not None and q.numel() else None,
             k.data_ptr() if k is not None and k.numel() else None, cu_ptr, b, off_ptr,
             start.data_ptr() if b else None, amount.data_ptr() if b else None, n, L, hq, hk, D,
-            float(theta), sec, int(rot_dim), _stream_ptr(dev, stream)), "cmr_rotate_qk_shift")
+            float(theta), sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)),
+            "cmr_rotate_qk_shift")
     return q, k
 
 
@@ -350,23 +364,35 @@ def rotate_qk_cache(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
 
 def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.Tensor,
               theta: float = 1e7, sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
-              stream: Optional[torch.cuda.Stream] = None):
+              stream: Optional[torch.cuda.Stream] = None,
+              device_status: Optional[torch.Tensor] = None):
     """cmr_rotate_qk, in place.  q: bf16 [L, N, hq, D] (or [N, hq, D]); k likewise
-    with hk heads; pos: int32 [3, N].  Returns (q, k)."""
+    with hk heads; pos: int32 [3, N]; device_status: optional int32 [1] on the
+    device (CMR_DEVICE_* bits).  Returns (q, k)."""
     _want(pos, "pos", torch.int32)
     dev = pos.device
     if pos.dim() != 2 or pos.shape[0] != 3:
         raise ValueError("pos must be [3, N]")
     n = pos.shape[1]
     L, hq, hk, D = _qk_shapes(q, k, dev, n)
+    st_ptr = _status_ptr(device_status, dev)
     sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
     with torch.cuda.device(dev):
         _check(lib().cmr_rotate_qk(q.data_ptr() if q is not None and q.numel() else None,
                                    k.data_ptr() if k is not None and k.numel() else None,
                                    pos.data_ptr() if n else None, n, L, hq, hk, D, float(theta),
-                                   sec, int(rot_dim), _stream_ptr(dev, stream)),
+                                   sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)),
                "cmr_rotate_qk")
     return q, k
+
+
+def rotate_qk_kernel(n_tokens: int, num_layers: int, hq: int, hk: int, head_dim: int = 256,
+                     rot_dim: int = 64) -> Optional[str]:
+    """Name of the kernel cmr_rotate_qk launches for these shapes (None if
+    there is nothing to launch or the shapes are invalid)."""
+    name = lib().cmr_rotate_qk_kernel(int(n_tokens), int(num_layers), int(hq), int(hk),
+                                      int(head_dim), int(rot_dim))
+    return None if name is None else name.decode()
 
 
 def copy_rotated_dims(dst: torch.Tensor, src: torch.Tensor, rot_dim: int = 64,

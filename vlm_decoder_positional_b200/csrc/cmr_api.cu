@@ -127,7 +127,7 @@ const char* cmr_status_string(cmr_status s) {
 
 const char* cmr_last_error_message(void) { return g_message; }
 
-int32_t cmr_version(void) { return 10300; }  // 1.3.0
+int32_t cmr_version(void) { return 20000; }  // 2.0.0
 
 cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
@@ -223,7 +223,7 @@ cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* start,
 cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
                          int32_t num_layers, int32_t hq, int32_t hk, int32_t head_dim,
                          double theta, const int32_t sections[3], int32_t rot_dim,
-                         cmr_stream_t stream) {
+                         int32_t* device_status, cmr_stream_t stream) {
   cmr::RotateArgs a;
   cmr::FreqTable table;
   cmr_status s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections,
@@ -231,7 +231,9 @@ cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
   if (s != CMR_OK || a.n_tokens == 0) return s;
   if (!pos) return fail(CMR_EINVAL, "pos is required");
   if ((s = check_device_ptr(pos, "pos")) != CMR_OK) return s;
+  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
   a.pos = pos;
+  a.status = device_status;
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
   return CMR_OK;
@@ -241,7 +243,8 @@ cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens, int3
                                const int32_t* pos_offset, const int32_t* start,
                                const int32_t* amount, int64_t n_tokens, int32_t num_layers,
                                int32_t hq, int32_t hk, int32_t head_dim, double theta,
-                               const int32_t sections[3], int32_t rot_dim, cmr_stream_t stream) {
+                               const int32_t sections[3], int32_t rot_dim,
+                               int32_t* device_status, cmr_stream_t stream) {
   cmr::RotateArgs a;
   cmr::FreqTable table;
   cmr_status s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections,
@@ -255,6 +258,8 @@ cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens, int3
   if (pos_offset && (s = check_device_ptr(pos_offset, "pos_offset")) != CMR_OK) return s;
   if ((s = check_device_ptr(start, "start")) != CMR_OK) return s;
   if ((s = check_device_ptr(amount, "amount")) != CMR_OK) return s;
+  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  a.status = device_status;
   a.cu = cu_seqlens;
   a.num_seqs = num_seqs;
   a.pos_offset = pos_offset;
@@ -263,6 +268,23 @@ cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqlens, int3
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk_shift launch");
   return CMR_OK;
+}
+
+const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, int32_t hq, int32_t hk,
+                                 int32_t head_dim, int32_t rot_dim) {
+  if (n_tokens <= 0 || num_layers <= 0 || hq < 0 || hk < 0 || hq + hk < 1) return nullptr;
+  if (head_dim <= 0 || head_dim % 8 != 0) return nullptr;
+  if (rot_dim < 16 || rot_dim % 16 != 0 || rot_dim > head_dim || rot_dim > 2 * cmr::kMaxFreqs)
+    return nullptr;
+  if ((static_cast<int64_t>(hq) + hk) * num_layers > INT32_MAX) return nullptr;
+  cmr::RotateArgs a{};
+  a.n_tokens = n_tokens;
+  a.num_layers = num_layers;
+  a.hq = hq;
+  a.hk = hk;
+  a.head_dim = head_dim;
+  a.rot_dim = rot_dim;
+  return cmr::rotate_qk_uses_staged(a) ? "rotate_qk_staged_kernel" : "rotate_qk_kernel";
 }
 
 cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v, const int32_t* cu_seqlens,

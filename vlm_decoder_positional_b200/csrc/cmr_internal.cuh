@@ -41,6 +41,7 @@ struct RotateArgs {
   int64_t n_tokens;
   int32_t num_layers;
   int32_t hq, hk, head_dim, rot_dim;
+  int32_t* status;         // optional device status word (staged kernel time-outs)
   int32_t units_per_head;  // rot_dim / 16: threads per token, 8 frequencies each
   int32_t job_groups;       // work items per token (set at launch)
   int32_t jobs_per_group;   // (layer, head) rows per work item
@@ -77,5 +78,15 @@ cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start
                                   cudaStream_t stream);
 
 cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream);
+
+// The TMA-staged rotate (rot_dim 64, one CTA per tile of tokens): whether it
+// can take these shapes, its tile count, and its launch (*launched false,
+// nothing enqueued, if the buffers cannot be described by tensor maps).
+bool staged_rotate_fits(const RotateArgs& args);
+// Whether launch_rotate_qk hands these shapes to the staged kernel.
+bool rotate_qk_uses_staged(const RotateArgs& args);
+int64_t staged_rotate_tiles(int64_t n_tokens);
+cudaError_t launch_rotate_qk_staged(const RotateArgs& args, const FreqTable& table,
+                                    cudaStream_t stream, bool* launched);
 
 }  // namespace cmr

@@ -40,6 +40,10 @@ using namespace rot;
 
 constexpr int kThreads = 128;
 constexpr int kOneShotRows = 16;  // rows per item from which a CTA serves one tile
+// From this many 8-token tiles on, rot_dim 64 goes to the TMA-staged kernel
+// (rotate_staged.cu); smaller batches (decode) keep this one, whose job groups
+// spread a token's rows over several threads.
+constexpr int64_t kMinStagedTiles = 1024;
 
 // kBatch head rows are in flight per thread; the launch bounds keep the
 // batch's registers within the occupancy each variant was tuned for.
@@ -217,7 +221,16 @@ Plan choose_plan(int rows_per_item) {
 
 }  // namespace
 
+bool rotate_qk_uses_staged(const RotateArgs& a) {
+  return staged_rotate_tiles(a.n_tokens) >= kMinStagedTiles && staged_rotate_fits(a);
+}
+
 cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream) {
+  if (rotate_qk_uses_staged(in)) {
+    bool launched = false;
+    const cudaError_t e = launch_rotate_qk_staged(in, table, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
   RotateArgs a = in;
   const bool from_shift = a.pos == nullptr;
   const int64_t items_per_cta = kThreads / a.units_per_head;
