@@ -88,6 +88,32 @@ __device__ __forceinline__ void store_4d(const CUtensorMap* map, uint32_t src, i
       : "memory");
 }
 
+// An L2 policy that marks the lines an access touches as first to evict.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// load_4d / store_4d with an L2 cache policy.
+__device__ __forceinline__ void load_4d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                             int x, int y, int z, int w, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void store_4d_hint(const CUtensorMap* map, uint32_t src, int x, int y,
+                                              int z, int w, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(map),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
