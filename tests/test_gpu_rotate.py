@@ -185,10 +185,10 @@ STAGED_MIN_TOKENS = 1024 * 8
 
 @pytest.mark.parametrize("n", [STAGED_MIN_TOKENS, STAGED_MIN_TOKENS + 1, STAGED_MIN_TOKENS + 7,
                                10001])
-@pytest.mark.parametrize("layers", [1, 3, 4, 5, 9])
+@pytest.mark.parametrize("layers", [1, 2, 3, 4, 5, 9])
 def test_rotate_staged_ragged_tiles_and_ring_wrap(cuda_device, n, layers):
-    # tiles of 8 tokens with a ragged last tile; 4, 5 and 9 layers wrap the
-    # 3-stage ring
+    # tiles of 8 tokens with a ragged last tile; 1 and 2 layers use a ring of
+    # that many stages; 4, 5 and 9 layers wrap the 3-stage ring
     assert cmr.rotate_qk_kernel(n, layers, 8, 2) == "rotate_qk_staged_kernel"
     g = torch.Generator(device=cuda_device).manual_seed(n + 100 * layers)
     q = torch.randn((layers, n, 8, 256), generator=g, device=cuda_device).to(torch.bfloat16)
