@@ -239,3 +239,39 @@ def test_shift_and_cache_forms_on_other_shapes(cuda_device, hq, hk, head_dim, ro
             got_v = vc[:, b_, :, :hi - lo].permute(0, 2, 1, 3)
             assert torch.equal(got_k.contiguous().view(torch.int16), ka[:, lo:hi].view(torch.int16))
             assert torch.equal(got_v.contiguous().view(torch.int16), v[:, lo:hi].view(torch.int16))
+
+
+@pytest.mark.parametrize("layers", [1, 3])
+def test_staged_shift_rotate_on_chunks_at_offsets(cuda_device, layers):
+    # second chunks of 4 prompts of 8,192 tokens, split so that two frames lie
+    # in the first chunks and two (one cut off by the prompt's end) in the
+    # second: 19,668 tokens, enough for the TMA-staged kernel.  The second
+    # chunks' state comes from cmr_positions_chunk at their offsets; the rotate
+    # derives every token's planes from it in the kernel.
+    dev = cuda_device
+    wl = inputs.make_batch([8192] * 4, [6, 2500, 5000, 8150], with_qk=False)
+    cut = [2000, 2600, 4000, 4500]
+    first = [wl.ids[wl.cu_seqlens[b]: wl.cu_seqlens[b] + cut[b]] for b in range(4)]
+    rest = [wl.ids[wl.cu_seqlens[b] + cut[b]: wl.cu_seqlens[b + 1]] for b in range(4)]
+    ids1, cu1 = inputs.pack(first)
+    ids2, cu2 = inputs.pack(rest)
+    _, s1, a1 = cmr.positions_chunk(t32(ids1, dev), t32(cu1, dev))
+    off = t32(np.array(cut), dev)
+    pos2, s, a = cmr.positions_chunk(t32(ids2, dev), t32(cu2, dev), pos_offset=off,
+                                     state=(s1, a1))
+    n2 = ids2.size
+    assert cmr.rotate_qk_kernel(n2, layers, 8, 2) == "rotate_qk_staged_kernel"
+    q = inputs.random_qk((layers, n2, 8, 256), 21, dev)
+    k = inputs.random_qk((layers, n2, 2, 256), 22, dev)
+    q_in, k_in = bits(q), bits(k)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    cmr.rotate_qk_shift(q, k, s, a, cu_seqlens=t32(cu2, dev), pos_offset=off,
+                        device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    whole = oracle.positions(wl.ids, wl.cu_seqlens, MARK)[0]
+    p = np.concatenate([whole[:, wl.cu_seqlens[b] + cut[b]: wl.cu_seqlens[b + 1]]
+                        for b in range(4)], axis=1)
+    np.testing.assert_array_equal(pos2.cpu().numpy(), p)
+    assert_bf16_close(bits(q), oracle.rotate_bf16(q_in, p), "staged chunk q")
+    assert_bf16_close(bits(k), oracle.rotate_bf16(k_in, p), "staged chunk k")

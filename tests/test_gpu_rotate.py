@@ -253,3 +253,16 @@ def test_staged_shift_form_matches_pos_form(cuda_device):
     assert int(status.item()) == 0
     assert torch.equal(wl.q.view(torch.int16), q2.view(torch.int16))
     assert torch.equal(wl.k.view(torch.int16), k2.view(torch.int16))
+
+
+@pytest.mark.parametrize("theta", [1e4, 5e8])
+def test_rotate_staged_other_theta_and_extreme_positions(cuda_device, theta):
+    g = torch.Generator(device=cuda_device).manual_seed(23)
+    n = 9000
+    assert cmr.rotate_qk_kernel(n, 1, 8, 2) == "rotate_qk_staged_kernel"
+    q = (torch.randn((1, n, 8, 256), generator=g, device=cuda_device) * 30).to(torch.bfloat16)
+    k = (torch.randn((1, n, 2, 256), generator=g, device=cuda_device) * 30).to(torch.bfloat16)
+    pos = torch.randint(-(2 ** 30), 2 ** 30, (3, n), generator=g, device=cuda_device,
+                        dtype=torch.int32)
+    pos[:, :3] = torch.tensor([0, 2 ** 31 - 1, -(2 ** 31)], dtype=torch.int32)
+    check_full(q, k, pos, theta, what=f"staged theta={theta}")
