@@ -73,8 +73,8 @@ typedef enum cmr_status {
  *   p == O + 65            -> (O, O+8, O+8)
  *   O + 65 < p < start     -> (O, O, O)
  *   p >= start             -> (p - amount) on all three planes
- * with start = O + 67 and amount = start - (O + 9) = 58 (port notes: "start =
- * i0 + 67", "amount = 58").  A prompt with no marker is text-only: start =
+ * with start = O + 67 and amount = start - (O + 9) = 58 (the port notes give
+ * start as i0 + 67 and amount as 58).  A prompt with no marker is text-only: start =
  * 2^30, amount = 0, every token (p, p, p).  Later markers in a prompt are
  * ordinary tokens.  Frames cut off by the end of a prompt keep the rows that
  * exist; start still reads O + 67.
@@ -110,8 +110,8 @@ CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
  * pos_offset[b] + m and
  *   CMR_RULE_CANVAS:    start = O + 67, amount = 58 (as cmr_positions);
  *   CMR_RULE_QWEN_VL:   start = O + 65, amount = 56 (port notes, CoreAIKit:
- *                       Qwen-VL's rule "would give + 64 and 56" from the
- *                       pads; </image> and "\n" then count as text after the
+ *                       Qwen-VL's rule shifts by 64 from the pads and by 56;
+ *                       </image> and "\n" then count as text after the
  *                       frame);
  *   CMR_RULE_PLANES_1D: no shift at all, state (2^30, 0) (the LiteRT card:
  *                       the runtime feeds plain 1-D positions).
@@ -140,8 +140,8 @@ CMR_API cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seq
                                        int32_t* device_status, cmr_stream_t stream);
 
 /* Planes of one new token per sequence, for decode and continuation (port
- * notes: "every generated token at p - amount"; canvas table row "everything
- * after the frame, generated tokens included").  Token b sits at absolute
+ * notes: generated tokens sit at p - amount; the canvas table's last row,
+ * after the frame, covers generated tokens too).  Token b sits at absolute
  * index p = cache_len[b] of its sequence, whose start / amount came from
  * cmr_positions.  As in the engine, which binds only start and amount, the
  * origin follows from amount = start - (O + 9); the token then gets the row of

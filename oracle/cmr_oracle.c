@@ -34,15 +34,15 @@
 #define GRID_SIDE 8
 #define GRID_ROWS 64
 /* <image> + 64 rows + </image> + "\n" with this chat template: start = O + 67
- * ([P1] "start = i0 + 67"; [P2] start = 73 for O = 6). */
+ * ([P1] writes it as i0 + 67; [P2] start = 73 for O = 6). */
 #define FRAME_TOKENS 67
-/* 9 = max(H, W) + 1 on the 8x8 grid ([P2] "amount = start - (O + 9)"). */
+/* 9 = max(H, W) + 1 on the 8x8 grid ([P2] defines amount as start minus O + 9). */
 #define CANVAS_SPAN 9
 /* Text-only prompts send start = 2^30 and amount = 0 ([P1], [P2]). */
 #define TEXT_ONLY_START (1 << 30)
 
 /* Rules the oracle can evaluate: the canvas rule and the pages' two red arms
- * ([P1] "Red arms in torch: amount + 1 fails 4/4 ..., 1-D planes fail 4/4"). */
+ * ([P1]: in torch, amount + 1 and 1-D planes each fail all four prompts). */
 #define RULE_CANVAS 0
 #define RULE_AMOUNT_PLUS_ONE 1
 #define RULE_PLANES_1D 2
@@ -157,7 +157,7 @@ int oracle_positions(const int32_t* ids, const int32_t* cu_seqlens,
 /* ------------------------------------------------------------------------ */
 
 /* Rules for the chunked form: the canvas rule; Qwen-VL's shift, which the
- * port notes' CoreAIKit section gives as "+ 64 and 56" from the index where the
+ * port notes' CoreAIKit section gives as 64 and 56 from the index where the
  * pads begin (start = O + 65, so </image> and "\n" count as text after the
  * frame, amount = start - (O + 9) = 56); and plain 1-D positions (the LiteRT
  * card: the runtime feeds plain 1-D positions). */
@@ -224,8 +224,8 @@ int oracle_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens,
 
 /* Decode / continuation: the token at absolute index p = cache_len[b] of
  * sequence b, with that sequence's start and amount.  Generated tokens sit at
- * p - amount on all three planes ([P1] "every generated token at p - amount";
- * [P2] "generated tokens included"). */
+ * p - amount on all three planes ([P1]; [P2]'s canvas table counts generated
+ * tokens in its last row). */
 int oracle_positions_step(const int32_t* cache_len, const int32_t* start,
                           const int32_t* amount, int32_t num_seqs,
                           int32_t* pos) {
@@ -242,7 +242,7 @@ int oracle_positions_step(const int32_t* cache_len, const int32_t* start,
 /* Frequencies                                                                */
 /* ------------------------------------------------------------------------ */
 
-/* Interleaved sections {T, H, W} ([P2] "interleaved sections [11, 11, 10]"):
+/* Interleaved sections {T, H, W} ([P2], "What it is": sections [11, 11, 10]):
  * frequency j belongs to H when j % 3 == 1 and j < 3*s_H, to W when
  * j % 3 == 2 and j < 3*s_W, and to T otherwise.  For {11, 11, 10} and 32
  * frequencies that is H if j%3==1 and j<33, W if j%3==2 and j<30.

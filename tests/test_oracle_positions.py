@@ -161,8 +161,8 @@ def test_malformed_cu_seqlens_rejected():
 
 @pytest.mark.parametrize("cfg", [1, 2, 3])
 def test_red_arms_fail_on_every_image_prompt(cfg):
-    # The pages' negative controls: "amount + 1" and "1-D planes" must give
-    # different planes; on text-only prompts every arm agrees.
+    # The pages' negative controls, the amount + 1 arm and the 1-D planes arm,
+    # must give different planes; on text-only prompts every arm agrees.
     wl = inputs.make_config(cfg, with_qk=False)
     green = oracle.positions(wl.ids, wl.cu_seqlens, MARK)[0]
     plus1 = oracle.positions(wl.ids, wl.cu_seqlens, MARK, rule="amount+1")[0]
