@@ -1,6 +1,6 @@
 // sm_100a primitives for kernels that stage tiles through shared memory with
 // the Tensor Memory Accelerator: mbarriers with bounded waits, tiled bulk
-// tensor loads and stores (no cluster multicast anywhere), the async-proxy
+// tensor loads and stores of this CTA's own boxes, the async-proxy
 // fence, and named barriers.  Inline PTX, written from the PTX ISA's
 // descriptions of mbarrier, cp.async.bulk.tensor and bar.
 #pragma once
