@@ -275,3 +275,47 @@ def test_staged_shift_rotate_on_chunks_at_offsets(cuda_device, layers):
     np.testing.assert_array_equal(pos2.cpu().numpy(), p)
     assert_bf16_close(bits(q), oracle.rotate_bf16(q_in, p), "staged chunk q")
     assert_bf16_close(bits(k), oracle.rotate_bf16(k_in, p), "staged chunk k")
+
+
+FIRST_CALL_IN_CAPTURE = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from vlm_decoder_positional_b200 import cmr, inputs
+dev = torch.device("cuda", 0)
+L, n = 2, 20000
+assert cmr.rotate_qk_kernel(n, L, 8, 2) == "rotate_qk_staged_kernel"
+q0 = inputs.random_qk((L, n, 8, 256), 3, dev)
+k0 = inputs.random_qk((L, n, 2, 256), 4, dev)
+pos = torch.randint(0, 40000, (3, n), dtype=torch.int32, device=dev)
+q, k = q0.clone(), k0.clone()
+status = torch.zeros(1, dtype=torch.int32, device=dev)
+torch.cuda.synchronize()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g):          # the process's first library call
+    cmr.rotate_qk(q, k, pos, device_status=status)
+q.copy_(q0); k.copy_(k0)
+g.replay()
+torch.cuda.synchronize()
+qe, ke = q0.clone(), k0.clone()
+cmr.rotate_qk(qe, ke, pos, device_status=status)
+torch.cuda.synchronize()
+assert int(status.item()) == 0
+assert torch.equal(q.view(torch.int16), qe.view(torch.int16))
+assert torch.equal(k.view(torch.int16), ke.view(torch.int16))
+print("ok")
+"""
+
+
+def test_first_call_of_a_process_inside_graph_capture(cuda_device, tmp_path):
+    # a fresh process whose very first library call is a staged rotate being
+    # captured into a CUDA graph: the launch path makes no call that a capture
+    # forbids, and the replay equals an eager launch bit for bit
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = tmp_path / "first_call.py"
+    script.write_text(FIRST_CALL_IN_CAPTURE)
+    out = subprocess.run([sys.executable, str(script), root], capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0 and out.stdout.strip().endswith("ok"), out.stderr[-2000:]

@@ -290,8 +290,11 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
   int64_t l2_bytes = 0;
   {
     std::lock_guard<std::mutex> lock(g_dev.mu);
+    // Only shapes whose ring exceeds the default 48 KB of dynamic shared
+    // memory need the opt-in (10 KB stages of 8 + 2 heads never do), so the
+    // common launch makes no attribute call, inside a graph capture or not.
     bool& done = g_dev.smem_set[dev & 63][from_shift ? 1 : 0];
-    if (!done) {
+    if (!done && smem > 48 * 1024) {
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(1024 + kStages * (kMaxStageBytes + 16)));
       if (e != cudaSuccess) return e;
