@@ -386,7 +386,8 @@ def run_ours(args):
         k_cache = torch.zeros((L, b, wl.hk, ctx, wl.head_dim), dtype=torch.bfloat16, device=dev)
         v_cache = torch.zeros_like(k_cache)
         rot_b = cache_bytes(wl.qk_tokens, L, wl.hq, wl.hk, wl.rot_dim, wl.head_dim)
-        kernel = "rotate_qk_cache_kernel"
+        kernel = cmr.rotate_qk_cache_kernel(wl.qk_tokens, L, wl.hq, wl.hk, wl.head_dim,
+                                            wl.rot_dim)
     if decode:
         # The prompts' (start, amount) come from their prefill, once; a decode
         # step is one launch that derives each new token's planes in the

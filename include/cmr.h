@@ -228,6 +228,16 @@ CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqle
 CMR_API const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, int32_t hq,
                                          int32_t hk, int32_t head_dim, int32_t rot_dim);
 
+/* The same for cmr_rotate_qk_cache: "rotate_qk_cache_staged_kernel" (TMA-staged,
+ * rot_dim 64, large batches, head_dim <= 256, K/V token rows a multiple of
+ * 128 B) or "rotate_qk_cache_kernel".  The staged kernel's first launch in a
+ * process needs more than the default shared memory; if that first launch is
+ * being captured into a CUDA graph, it takes rotate_qk_cache_kernel.  NULL when
+ * the shapes are invalid or there is nothing to launch. */
+CMR_API const char* cmr_rotate_qk_cache_kernel(int64_t n_tokens, int32_t num_layers,
+                                               int32_t hq, int32_t hk, int32_t head_dim,
+                                               int32_t rot_dim);
+
 /* Rotate Q in place and write each token's rotated K row and its V row into
  * a KV cache, in one pass: the step after the rotation in the full-attention
  * layers (HF card mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides

@@ -29,6 +29,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
                           "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache", "cmr_rotate_qk_kernel",
+                          "cmr_rotate_qk_cache_kernel",
                           "cmr_copy_rotated_dims", "cmr_status_string",
                           "cmr_last_error_message", "cmr_version"}
     assert set(names) == set(cmr.SIGNATURES)
@@ -172,3 +173,21 @@ def test_kernel_query_names_the_path_each_shape_takes(lib):
                 (10, 1, 8, 2, 250, 64), (10, 1, 8, 2, 256, 24), (10, 1, 8, 2, 32, 64),
                 (10, 80000, 30000, 2, 256, 64), (-1, 1, 8, 2, 256, 64)]:
         assert name(*bad) is None, bad
+
+
+def test_cache_kernel_query(lib):
+    def name(*a):
+        r = lib.cmr_rotate_qk_cache_kernel(*a)
+        return None if r is None else r.decode()
+    staged, regs = "rotate_qk_cache_staged_kernel", "rotate_qk_cache_kernel"
+    assert name(262144, 6, 8, 2, 256, 64) == staged
+    assert name(8185, 1, 8, 2, 256, 64) == staged
+    assert name(8184, 1, 8, 2, 256, 64) == regs
+    assert name(1024, 6, 8, 2, 256, 64) == regs           # decode
+    assert name(262144, 6, 8, 2, 256, 128) == regs         # rot_dim other than 64
+    assert name(262144, 6, 8, 0, 256, 64) == regs          # no K/V: nothing to cache
+    assert name(262144, 6, 16, 4, 256, 64) == regs         # 48-KB stage: too big
+    assert name(262144, 6, 8, 2, 512, 64) == regs          # head_dim over one box
+    assert name(262144, 6, 8, 1, 72, 64) == regs           # 144-B token rows
+    assert name(262144, 6, 8, 2, 64, 64) == staged
+    assert name(0, 6, 8, 2, 256, 64) is None

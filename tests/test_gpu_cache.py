@@ -129,3 +129,54 @@ def test_cache_path_matches_shift_path_bit_for_bit(cuda_device):
     assert torch.equal(kc_tokens.view(torch.int16), k2.view(torch.int16))
     vc_tokens = vc.permute(0, 1, 3, 2, 4).reshape(1, 64 * 4096, 2, 256)
     assert torch.equal(vc_tokens.view(torch.int16), v.view(torch.int16))
+
+
+# ---- the TMA-staged cache kernel (rot_dim 64, from 1024 tiles of 8 tokens) ----
+
+@pytest.mark.parametrize("layers", [1, 2, 4])
+def test_staged_prefill_into_permuted_slots_with_out_of_range_tokens(cuda_device, layers):
+    # 16,400 tokens in 4 prompts (a ragged last tile), slots permuted inside a
+    # 5-sequence cache whose context (4,100) leaves the last 11 tokens of the
+    # 4,111-token prompt outside: those write no K/V and set the status bit
+    dev = cuda_device
+    wl = inputs.make_batch([4100, 4096, 4111, 4093], [6, 17, 3000, 4080], num_layers=layers,
+                           with_qk=False)
+    n = wl.n_tokens
+    assert cmr.rotate_qk_cache_kernel(n, layers, 8, 2) == "rotate_qk_cache_staged_kernel"
+    cu = t32(wl.cu_seqlens, dev)
+    _, s, a = cmr.positions(t32(wl.ids, dev), cu)
+    q = inputs.random_qk((layers, n, 8, 256), 31, dev)
+    k = inputs.random_qk((layers, n, 2, 256), 32, dev)
+    v = inputs.random_qk((layers, n, 2, 256), 33, dev)
+    kc = sentinel_cache((layers, 5, 2, 4100, 256), dev)
+    vc = sentinel_cache((layers, 5, 2, 4100, 256), dev)
+    run_and_compare(q, k, v, s, a, kc, vc, cu=cu, slot=t32([2, 0, 4, 1], dev),
+                    status_want=cmr.CMR_DEVICE_CACHE_RANGE)
+
+
+def test_staged_kernels_are_the_ones_that_run(cuda_device):
+    # the kernel names the library reports are the kernels the profiler sees
+    from torch.profiler import ProfilerActivity, profile
+    dev = cuda_device
+    wl = inputs.make_batch([4100, 4100], [6, 17], num_layers=2, with_qk=False)
+    n = wl.n_tokens
+    cu = t32(wl.cu_seqlens, dev)
+    pos, s, a = cmr.positions(t32(wl.ids, dev), cu)
+    q = inputs.random_qk((2, n, 8, 256), 41, dev)
+    k = inputs.random_qk((2, n, 2, 256), 42, dev)
+    v = inputs.random_qk((2, n, 2, 256), 43, dev)
+    kc = sentinel_cache((2, 2, 2, 4100, 256), dev)
+    vc = sentinel_cache((2, 2, 2, 4100, 256), dev)
+    cmr.rotate_qk_cache(q, k, v, s, a, kc, vc, cu_seqlens=cu)   # first launch outside capture
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        cmr.rotate_qk(q, k, pos)
+        cmr.rotate_qk_cache(q, k, v, s, a, kc, vc, cu_seqlens=cu)
+        q1, k1 = q[:1, :512].contiguous(), k[:1, :512].contiguous()
+        cmr.rotate_qk(q1, k1, pos[:, :512].contiguous())
+        torch.cuda.synchronize()
+    names = " ".join(e.name for e in prof.events())
+    for kernel in (cmr.rotate_qk_kernel(n, 2, 8, 2), cmr.rotate_qk_cache_kernel(n, 2, 8, 2),
+                   cmr.rotate_qk_kernel(512, 1, 8, 2)):
+        assert kernel + "<" in names or kernel + "(" in names, (kernel, names[:2000])
+    assert "rotate_qk_staged_kernel" in names and "rotate_qk_cache_staged_kernel" in names

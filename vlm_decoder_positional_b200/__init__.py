@@ -8,11 +8,12 @@ Both run hand-written sm_100a kernels in libcmr.so through its C ABI
 """
 from .cmr import (CMR_DEVICE_BAD_CU_SEQLENS, CMR_ECUDA, CMR_EINVAL, CMR_EUNSUPPORTED, CMR_OK,
                   CMR_DEVICE_CACHE_RANGE, CMR_DEVICE_WAIT_TIMEOUT, CmrError, lib, positions, positions_chunk,
-                  positions_step, rotate_qk, rotate_qk_cache, rotate_qk_kernel, rotate_qk_shift,
+                  positions_step, rotate_qk, rotate_qk_cache, rotate_qk_cache_kernel, rotate_qk_kernel,
+                  rotate_qk_shift,
                   version)
 
 __all__ = ["positions", "positions_chunk", "positions_step", "rotate_qk", "rotate_qk_shift",
-           "rotate_qk_kernel",
+           "rotate_qk_kernel", "rotate_qk_cache_kernel",
            "rotate_qk_cache", "CMR_DEVICE_CACHE_RANGE", "CMR_DEVICE_WAIT_TIMEOUT",
            "lib", "version", "CmrError",
            "CMR_OK", "CMR_EINVAL", "CMR_ECUDA", "CMR_EUNSUPPORTED", "CMR_DEVICE_BAD_CU_SEQLENS"]

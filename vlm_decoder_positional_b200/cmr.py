@@ -53,6 +53,9 @@ SIGNATURES = {
                                      _i32p, ctypes.c_void_p]),
     "cmr_rotate_qk_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
+    "cmr_rotate_qk_cache_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32,
+                                                     ctypes.c_int32, ctypes.c_int32,
+                                                     ctypes.c_int32, ctypes.c_int32]),
     "cmr_copy_rotated_dims": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                              ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_void_p]),
@@ -392,6 +395,15 @@ def rotate_qk_kernel(n_tokens: int, num_layers: int, hq: int, hk: int, head_dim:
     there is nothing to launch or the shapes are invalid)."""
     name = lib().cmr_rotate_qk_kernel(int(n_tokens), int(num_layers), int(hq), int(hk),
                                       int(head_dim), int(rot_dim))
+    return None if name is None else name.decode()
+
+
+def rotate_qk_cache_kernel(n_tokens: int, num_layers: int, hq: int, hk: int,
+                           head_dim: int = 256, rot_dim: int = 64) -> Optional[str]:
+    """Name of the kernel cmr_rotate_qk_cache launches for these shapes (None if
+    there is nothing to launch or the shapes are invalid)."""
+    name = lib().cmr_rotate_qk_cache_kernel(int(n_tokens), int(num_layers), int(hq), int(hk),
+                                            int(head_dim), int(rot_dim))
     return None if name is None else name.decode()
 
 

@@ -287,6 +287,21 @@ const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, int32_t h
   return cmr::rotate_qk_uses_staged(a) ? "rotate_qk_staged_kernel" : "rotate_qk_kernel";
 }
 
+const char* cmr_rotate_qk_cache_kernel(int64_t n_tokens, int32_t num_layers, int32_t hq,
+                                       int32_t hk, int32_t head_dim, int32_t rot_dim) {
+  if (cmr_rotate_qk_kernel(n_tokens, num_layers, hq, hk, head_dim, rot_dim) == nullptr)
+    return nullptr;
+  cmr::RotateArgs a{};
+  a.n_tokens = n_tokens;
+  a.num_layers = num_layers;
+  a.hq = hq;
+  a.hk = hk;
+  a.head_dim = head_dim;
+  a.rot_dim = rot_dim;
+  return cmr::rotate_qk_cache_uses_staged(a) ? "rotate_qk_cache_staged_kernel"
+                                             : "rotate_qk_cache_kernel";
+}
+
 cmr_status cmr_rotate_qk_cache(void* q, const void* k, const void* v, const int32_t* cu_seqlens,
                                int32_t num_seqs, const int32_t* pos_offset, const int32_t* start,
                                const int32_t* amount, int64_t n_tokens, int32_t num_layers,

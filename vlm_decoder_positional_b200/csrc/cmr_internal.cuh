@@ -1,6 +1,7 @@
 // Internal declarations shared by the kernels and the C-ABI layer of libcmr.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -67,6 +68,14 @@ struct CacheArgs {
 cudaError_t launch_rotate_qk_cache(const CacheArgs& args, const FreqTable& table,
                                    cudaStream_t stream);
 
+// The TMA-staged rotate + KV-cache write (rot_dim 64, large batches): whether
+// launch_rotate_qk_cache hands these shapes to it, and its launch (*launched
+// false, nothing enqueued, when tensor maps cannot describe the buffers or the
+// first launch falls inside a stream capture).
+bool rotate_qk_cache_uses_staged(const RotateArgs& args);
+cudaError_t launch_rotate_qk_cache_staged(const CacheArgs& args, const FreqTable& table,
+                                          cudaStream_t stream, bool* launched);
+
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                              int64_t n_tokens, int32_t image_token_id, int32_t rule,
                              const int32_t* pos_offset, const int32_t* in_start,
@@ -78,6 +87,15 @@ cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start
                                   cudaStream_t stream);
 
 cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream);
+
+// TMA tensor map of a bf16 tensor: dims[0] is contiguous, strides_bytes[i] is
+// the byte stride of dims[i + 1] (any order), box[i] the box extent per dim.
+// False (and *map untouched) when the driver cannot encode it.
+bool encode_bf16_tensor_map(CUtensorMap* map, void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box,
+                            bool swizzle_128b);
+// L2 size of the current device in bytes (cached; 0 if it cannot be read).
+int64_t device_l2_bytes();
 
 // The TMA-staged rotate (rot_dim 64, one CTA per tile of tokens): whether it
 // can take these shapes, its tile count, and its launch (*launched false,

@@ -198,6 +198,11 @@ cudaError_t resident_ctas(int* total) {
 
 cudaError_t launch_rotate_qk_cache(const CacheArgs& in, const FreqTable& table,
                                    cudaStream_t stream) {
+  if (rotate_qk_cache_uses_staged(in.r)) {
+    bool launched = false;
+    const cudaError_t e = launch_rotate_qk_cache_staged(in, table, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
+  }
   CacheArgs ca = in;
   RotateArgs& a = ca.r;
   int max_ctas = 0;

@@ -203,42 +203,16 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---- host side ----
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// cuTensorMapEncodeTiled from the driver (the runtime is linked statically, so
-// the driver entry point is looked up once at run time).
-EncodeTiledFn encoder() {
-  static std::once_flag once;
-  static EncodeTiledFn fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-    else
-      cudaGetLastError();
-  });
-  return fn;
-}
-
 // Tensor map of x [L, N, heads, head_dim] bf16 seen as {d, t, h, l}, with a
 // {64, kTileTokens, heads, 1} box, 128-B swizzle.
-bool encode_map(EncodeTiledFn enc, CUtensorMap* map, void* base, int64_t n_tokens, int heads,
-                int layers, int head_dim) {
-  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(n_tokens),
-                              static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(layers)};
-  const cuuint64_t strides[3] = {row * heads, row, row * heads * static_cast<cuuint64_t>(n_tokens)};
-  const cuuint32_t box[4] = {kStagedRotDim, kTileTokens, static_cast<cuuint32_t>(heads), 1};
-  const cuuint32_t unit[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, unit,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+bool encode_map(CUtensorMap* map, void* base, int64_t n_tokens, int heads, int layers,
+                int head_dim) {
+  const uint64_t row = static_cast<uint64_t>(head_dim) * 2;
+  const uint64_t dims[4] = {static_cast<uint64_t>(head_dim), static_cast<uint64_t>(n_tokens),
+                            static_cast<uint64_t>(heads), static_cast<uint64_t>(layers)};
+  const uint64_t strides[3] = {row * heads, row, row * heads * static_cast<uint64_t>(n_tokens)};
+  const uint32_t box[4] = {kStagedRotDim, kTileTokens, static_cast<uint32_t>(heads), 1};
+  return encode_bf16_tensor_map(map, base, 4, dims, strides, box, true);
 }
 
 using StagedFn = void (*)(CUtensorMap, CUtensorMap, StagedArgs, FreqTable);
@@ -246,7 +220,6 @@ using StagedFn = void (*)(CUtensorMap, CUtensorMap, StagedArgs, FreqTable);
 struct DeviceCache {
   std::mutex mu;
   bool smem_set[64][2] = {};
-  int64_t l2_bytes[64] = {};
 };
 DeviceCache g_dev;
 
@@ -268,12 +241,10 @@ int64_t staged_rotate_tiles(int64_t n_tokens) { return (n_tokens + kTileTokens -
 cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
                                     cudaStream_t stream, bool* launched) {
   *launched = false;
-  EncodeTiledFn enc = encoder();
-  if (enc == nullptr) return cudaSuccess;
   CUtensorMap q_map{}, k_map{};
-  if (a.hq > 0 && !encode_map(enc, &q_map, a.q, a.n_tokens, a.hq, a.num_layers, a.head_dim))
+  if (a.hq > 0 && !encode_map(&q_map, a.q, a.n_tokens, a.hq, a.num_layers, a.head_dim))
     return cudaSuccess;
-  if (a.hk > 0 && !encode_map(enc, &k_map, a.k, a.n_tokens, a.hk, a.num_layers, a.head_dim))
+  if (a.hk > 0 && !encode_map(&k_map, a.k, a.n_tokens, a.hk, a.num_layers, a.head_dim))
     return cudaSuccess;
   StagedArgs sa;
   sa.r = a;
@@ -287,7 +258,6 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int64_t l2_bytes = 0;
   {
     std::lock_guard<std::mutex> lock(g_dev.mu);
     // Only shapes whose ring exceeds the default 48 KB of dynamic shared
@@ -295,19 +265,19 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
     // common launch makes no attribute call, inside a graph capture or not.
     bool& done = g_dev.smem_set[dev & 63][from_shift ? 1 : 0];
     if (!done && smem > 48 * 1024) {
+      // a capture may forbid the attribute call: that first launch takes the
+      // register kernel instead
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      e = cudaStreamIsCapturing(stream, &cap);
+      if (e != cudaSuccess) return e;
+      if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(1024 + kStages * (kMaxStageBytes + 16)));
       if (e != cudaSuccess) return e;
       done = true;
     }
-    if (g_dev.l2_bytes[dev & 63] == 0) {
-      int l2 = 0;
-      e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
-      if (e != cudaSuccess) return e;
-      g_dev.l2_bytes[dev & 63] = l2 > 0 ? l2 : 1;
-    }
-    l2_bytes = g_dev.l2_bytes[dev & 63];
   }
+  const int64_t l2_bytes = device_l2_bytes();
   // L2 policy.  A launch that moves a few L2 sizes or less ends with most of
   // its rows still dirty in L2, and whatever reads them next competes with
   // their write-back (measured: the device-to-host copies of a 16,384-token,

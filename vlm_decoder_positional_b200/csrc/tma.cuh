@@ -114,6 +114,26 @@ __device__ __forceinline__ void store_4d_hint(const CUtensorMap* map, uint32_t s
       : "memory");
 }
 
+// 5-D tiled store of one box from shared memory (bulk async-group), plain and
+// with an L2 cache policy.
+__device__ __forceinline__ void store_5d(const CUtensorMap* map, uint32_t src, int x, int y, int z,
+                                         int w, int v) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
+          map),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void store_5d_hint(const CUtensorMap* map, uint32_t src, int x, int y,
+                                              int z, int w, int v, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.global.shared::cta.bulk_group.L2::cache_hint"
+      " [%0, {%2, %3, %4, %5, %6}], [%1], %7;" ::"l"(map),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w), "r"(v), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
