@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_staged.cu",
                   "vlm_decoder_positional_b200/csrc/tma.cuh",
+                  "vlm_decoder_positional_b200/csrc/tensor_map.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_common.cuh",
                   "vlm_decoder_positional_b200/csrc/canvas.cuh",
                   "vlm_decoder_positional_b200/csrc/cmr_internal.cuh",
