@@ -249,7 +249,9 @@ CMR_API const char* cmr_rotate_qk_cache_kernel(int64_t n_tokens, int32_t num_lay
  *   v_cache[l, slot, h, p, :] = V[l, t, h, :]
  * with slot = cache_slot[b] (or b when cache_slot is NULL).  K and V are not
  * modified.  A token whose p or slot falls outside the cache writes no K/V row
- * and ORs CMR_DEVICE_CACHE_RANGE into device_status.
+ * and ORs CMR_DEVICE_CACHE_RANGE into device_status.  Large batches with
+ * rot_dim 64 run a TMA-staged kernel (cmr_rotate_qk_cache_kernel says which);
+ * the result is the same bit for bit either way.
  *
  *   q                  device bf16 [num_layers, n_tokens, hq, head_dim], rotated in place
  *   k, v               device bf16 [num_layers, n_tokens, hk, head_dim], read only
