@@ -1,4 +1,7 @@
-// Fused cos/sin + rotate-half M-RoPE of Q and K, in place, on sm_100a.
+// Fused cos/sin + rotate-half M-RoPE of Q and K, in place, on sm_100a, with
+// the rows held in registers: the kernel for decode-sized batches and for
+// rot_dim other than 64 (larger rot_dim-64 batches go to the TMA-staged kernel
+// of rotate_staged.cu, which launch_rotate_qk below picks; same bits).
 // The planes come from pos [3, N] (cmr_rotate_qk) or are derived in the kernel
 // from each prompt's (start, amount) state (cmr_rotate_qk_shift).
 //

@@ -1,5 +1,8 @@
 // Rotate Q in place and write the rotated K and the V rows of the same tokens
-// into a KV cache, in one pass, on sm_100a.
+// into a KV cache, in one pass, on sm_100a, with the rows held in registers:
+// the kernel for decode-sized batches and other shapes (larger rot_dim-64
+// batches go to rotate_cache_staged.cu, which launch_rotate_qk_cache below
+// picks; same bits).
 //
 // The cache is the engine's keyCache / valueCache of the HF card
 // mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI ("How the VLM rides the text-only
