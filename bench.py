@@ -538,6 +538,12 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
         h_start.copy_(s)
         h_amount.copy_(a)
         h_cl = torch.from_numpy(wl.cache_len).pin_memory()
+        # device buffers for the step; only the rotated dims of each head row
+        # cross PCIe (cmr_copy_rotated_dims), as in the prefill pipeline
+        d_q, d_k = torch.empty_like(wl.q), torch.empty_like(wl.k)
+        d_cl = torch.empty_like(h_cl, device=dev)
+        d_start = torch.empty_like(h_start, device=dev)
+        d_amount = torch.empty_like(h_amount, device=dev)
 
     else:
         # prefill: chunks of whole prompts through a ring of device buffers,
@@ -549,15 +555,17 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
 
     def step():
         if decode:
-            q = h_q.to(dev, non_blocking=True)
-            k = h_k.to(dev, non_blocking=True)
-            cl = h_cl.to(dev, non_blocking=True)
-            start = h_start.to(dev, non_blocking=True)
-            amount = h_amount.to(dev, non_blocking=True)
-            cmr.rotate_qk_shift(q, k, start, amount, pos_offset=cl, theta=wl.theta,
+            for l in range(wl.num_layers):
+                cmr.copy_rotated_dims(d_q[l], h_q[l], wl.rot_dim, stream)
+                cmr.copy_rotated_dims(d_k[l], h_k[l], wl.rot_dim, stream)
+            d_cl.copy_(h_cl, non_blocking=True)
+            d_start.copy_(h_start, non_blocking=True)
+            d_amount.copy_(h_amount, non_blocking=True)
+            cmr.rotate_qk_shift(d_q, d_k, d_start, d_amount, pos_offset=d_cl, theta=wl.theta,
                                 sections=wl.sections, rot_dim=wl.rot_dim)
-            h_q.copy_(q, non_blocking=True)
-            h_k.copy_(k, non_blocking=True)
+            for l in range(wl.num_layers):
+                cmr.copy_rotated_dims(h_q[l], d_q[l], wl.rot_dim, stream)
+                cmr.copy_rotated_dims(h_k[l], d_k[l], wl.rot_dim, stream)
         else:
             pipe.run(h_ids, wl.cu_seqlens, h_q, h_k, h_pos, h_start, h_amount, wl.theta,
                      wl.sections, wl.rot_dim, wl.image_token_id, chunk_tokens=chunk)
@@ -573,18 +581,19 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
     z.record(stream)
     torch.cuda.synchronize(dev)
     ms = shard.max_over_ranks(a.elapsed_time(z), dist, dev)
+    rot = (h_q.numel() + h_k.numel()) // wl.head_dim * wl.rot_dim * 2
     if decode:
-        h2d = h_q.numel() * 2 + h_k.numel() * 2 + 12 * wl.num_seqs
-        d2h = h_q.numel() * 2 + h_k.numel() * 2
+        h2d = rot + 12 * wl.num_seqs
+        d2h = rot
     else:
         # the pipeline moves only the rotated dims of every head row
-        rot = (h_q.numel() + h_k.numel()) // wl.head_dim * wl.rot_dim * 2
         h2d = h_ids.numel() * 4 + h_cu.numel() * 4 + rot
         d2h = rot + h_pos.numel() * 4 + 8 * wl.num_seqs
     return {"value": tokens_all * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": ms / steps,
-            "path": ("pinned host -> cmr.rotate_qk_shift -> pinned host" if decode else
+            "path": ("pinned host -> rotated dims in (pitched copies), cmr.rotate_qk_shift, "
+                     "rotated dims out -> pinned host" if decode else
                      "pinned host -> HostPipeline: chunks of whole prompts, rotated dims in "
                      "(pitched copies), cmr.positions + cmr.rotate_qk, rotated dims out, on "
                      "three streams -> pinned host")}
