@@ -37,6 +37,12 @@ static int host_checks(void) {
   CHECK(cmr_positions_chunk(fake, fake, 1, 10, 248078, 7, NULL, NULL, NULL, fake, fake, fake,
                             NULL, NULL) == CMR_EINVAL);
   CHECK(cmr_copy_rotated_dims(fake, fake, 4, 64, 128, 0, NULL) == CMR_EINVAL);
+  /* which kernel a shape runs: pure host logic */
+  CHECK(strcmp(cmr_rotate_qk_kernel(262144, 6, 8, 2, 256, 64), "rotate_qk_staged_kernel") == 0);
+  CHECK(strcmp(cmr_rotate_qk_kernel(1024, 6, 8, 2, 256, 64), "rotate_qk_kernel") == 0);
+  CHECK(strcmp(cmr_rotate_qk_cache_kernel(262144, 6, 8, 2, 256, 64),
+               "rotate_qk_cache_staged_kernel") == 0);
+  CHECK(cmr_rotate_qk_kernel(0, 6, 8, 2, 256, 64) == NULL);
   printf("host ok\n");
   return 0;
 }
