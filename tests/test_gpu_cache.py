@@ -180,3 +180,51 @@ def test_staged_kernels_are_the_ones_that_run(cuda_device):
                    cmr.rotate_qk_kernel(512, 1, 8, 2)):
         assert kernel + "<" in names or kernel + "(" in names, (kernel, names[:2000])
     assert "rotate_qk_staged_kernel" in names and "rotate_qk_cache_staged_kernel" in names
+
+
+CACHE_FIRST_CALL_IN_CAPTURE = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+from vlm_decoder_positional_b200 import cmr, inputs
+dev = torch.device("cuda", 0)
+wl = inputs.make_batch([4100, 4100], [6, 17], num_layers=3, with_qk=False)
+n = wl.n_tokens
+assert cmr.rotate_qk_cache_kernel(n, 3, 8, 2) == "rotate_qk_cache_staged_kernel"
+cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+s = torch.tensor([73, 84], dtype=torch.int32, device=dev)
+a = torch.tensor([58, 58], dtype=torch.int32, device=dev)
+q0 = inputs.random_qk((3, n, 8, 256), 51, dev)
+k = inputs.random_qk((3, n, 2, 256), 52, dev)
+v = inputs.random_qk((3, n, 2, 256), 53, dev)
+def fresh():
+    kc = torch.zeros((3, 2, 2, 4100, 256), dtype=torch.bfloat16, device=dev)
+    return q0.clone(), kc, torch.zeros_like(kc)
+q1, kc1, vc1 = fresh()
+torch.cuda.synchronize()
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g):   # the process's first library call: the staged kernel would
+    cmr.rotate_qk_cache(q1, k, v, s, a, kc1, vc1, cu_seqlens=cu)   # need an attribute call
+g.replay()
+q2, kc2, vc2 = fresh()
+cmr.rotate_qk_cache(q2, k, v, s, a, kc2, vc2, cu_seqlens=cu)       # eager: staged kernel
+torch.cuda.synchronize()
+for x, y in ((q1, q2), (kc1, kc2), (vc1, vc2)):
+    assert torch.equal(x.view(torch.int16), y.view(torch.int16))
+print("ok")
+"""
+
+
+def test_cache_form_first_call_inside_graph_capture(cuda_device, tmp_path):
+    # a fresh process whose first library call is a staged-size cache form
+    # being captured: the launch falls back to the register kernel (the staged
+    # one needs a shared-memory opt-in first), and its replay equals the eager
+    # staged kernel's result bit for bit
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    script = tmp_path / "cache_first_call.py"
+    script.write_text(CACHE_FIRST_CALL_IN_CAPTURE)
+    out = subprocess.run([sys.executable, str(script), root], capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0 and out.stdout.strip().endswith("ok"), out.stderr[-2000:]
