@@ -16,6 +16,10 @@ def test_algorithmic_bytes_match_the_hand_count():
     assert bench.rotate_bytes(1, 1, 8, 2, 64) == 2560 + 12
     assert bench.rotate_bytes(262144, 6, 8, 2, 64) == 4_026_531_840 + 3_145_728
     assert bench.positions_bytes(262144, 32) == 262144 * 16 + 32 * 12
+    # rotate + KV cache, 8 Q + 2 KV heads of 256: Q's 64 dims read and written
+    # (2,048 B), K and V rows read (2,048 B), their cache rows written (2,048 B)
+    assert bench.cache_bytes(1, 1, 8, 2, 64, 256) == 6144
+    assert bench.cache_bytes(262144, 6, 8, 2, 64, 256) == 9_663_676_416
 
 
 def test_traffic_record_is_tied_to_the_kernel_source_and_workload():
