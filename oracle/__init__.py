@@ -43,6 +43,10 @@ def _load():
                                                ctypes.c_int32, ctypes.c_int32, i32p, i32p, i32p,
                                                i32p, i32p, i32p]
         lib.oracle_positions_chunk.restype = ctypes.c_int
+        lib.oracle_positions_frames.argtypes = [i32p, i32p, ctypes.c_int32, ctypes.c_int64,
+                                                ctypes.c_int32, ctypes.c_int32, i32p, i32p,
+                                                i32p]
+        lib.oracle_positions_frames.restype = ctypes.c_int
         lib.oracle_positions_step.argtypes = [i32p, i32p, i32p, ctypes.c_int32, i32p]
         lib.oracle_positions_step.restype = ctypes.c_int
         lib.oracle_freq_planes.argtypes = [ctypes.c_int32, i32p, i32p]
@@ -116,6 +120,25 @@ def positions_chunk(ids, cu_seqlens, image_token_id=248078, rule="canvas", pos_o
                                     _i32(start)[1], _i32(amount)[1])
     if st != 0:
         raise OracleError("oracle_positions_chunk: invalid arguments")
+    return pos, start, amount
+
+
+def positions_frames(ids, cu_seqlens, image_token_id=248078, grid_side=8):
+    """Planes of a packed batch in which every <image> marker opens a frame of
+    grid_side^2 + 3 tokens (the multi-frame reading of cmr_oracle.c).  Returns
+    (pos [3, N], start [B], amount [B])."""
+    lib = _load()
+    ids, ids_p = _i32(ids)
+    cu, cu_p = _i32(cu_seqlens)
+    n = int(ids.shape[0])
+    b = int(cu.shape[0]) - 1
+    pos = np.zeros((3, n), dtype=np.int32)
+    start = np.zeros(max(b, 0), dtype=np.int32)
+    amount = np.zeros(max(b, 0), dtype=np.int32)
+    st = lib.oracle_positions_frames(ids_p, cu_p, b, n, int(image_token_id), int(grid_side),
+                                     _i32(pos)[1], _i32(start)[1], _i32(amount)[1])
+    if st != 0:
+        raise OracleError("oracle_positions_frames: invalid arguments")
     return pos, start, amount
 
 

@@ -222,6 +222,99 @@ int oracle_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens,
   return ORC_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Several frames per prompt, any grid side                                   */
+/* ------------------------------------------------------------------------ */
+
+/* The pages print the canvas only for one 448x448 thumbnail per prompt (an
+ * 8x8 grid); the MNN card says its canvas positions were also checked on
+ * sliced and multi-image prompts, and the thumbnail's own numbers fix the
+ * structure: a frame lies on a canvas anchored at the text position where it
+ * starts, and the text after it resumes one past the largest coordinate the
+ * frame used ([P2]: 9 = max(H, W) + 1).  The reading taken here, for a grid of
+ * side s (8 for the thumbnail, 16 for a 4x-larger grid):
+ *   - a running counter c starts at 0; a text token gets (c, c, c) and c
+ *     advances by 1;
+ *   - every <image> marker opens a frame of s*s + 3 tokens laid at the
+ *     counter's value f: <image> (f, f-1, f-1); image row k (k < s*s, row-
+ *     major on the s x s grid) (f, f + k/s, f + k%s); </image> (f, f+s, f+s);
+ *     the "\n" (f, f, f); the counter moves to f + s + 1, one past the
+ *     frame's largest coordinate;
+ *   - a frame cut short by the next marker or by the end of the prompt keeps
+ *     the rows that exist, and the counter still stands at f + s + 1 after it
+ *     (as a truncated thumbnail keeps start = O + 67).
+ * With one marker and s = 8 this is the canvas rule (oracle_positions).
+ * State after the prompt: start = (index of the last marker) + s*s + 3, and
+ * amount such that the text from start on sits at p - amount; text-only
+ * prompts (2^30, 0).  Parity with the pages is unpinned beyond the one-frame
+ * case: they print no multi-frame values. */
+int oracle_positions_frames(const int32_t* ids, const int32_t* cu_seqlens,
+                            int32_t num_seqs, int64_t n_tokens,
+                            int32_t image_token_id, int32_t grid_side,
+                            int32_t* pos, int32_t* start_out,
+                            int32_t* amount_out) {
+  if (num_seqs < 0 || n_tokens < 0 || grid_side < 1 || grid_side > 128)
+    return ORC_EINVAL;
+  if (num_seqs == 0) return n_tokens == 0 ? ORC_OK : ORC_EINVAL;
+  if (cu_seqlens[0] != 0 || (int64_t)cu_seqlens[num_seqs] != n_tokens)
+    return ORC_EINVAL;
+  for (int32_t b = 0; b < num_seqs; ++b)
+    if (cu_seqlens[b + 1] < cu_seqlens[b]) return ORC_EINVAL;
+
+  const int64_t s = grid_side;
+  const int64_t frame_len = s * s + 3;
+  for (int32_t b = 0; b < num_seqs; ++b) {
+    const int64_t first = cu_seqlens[b];
+    const int64_t len = (int64_t)cu_seqlens[b + 1] - first;
+    int64_t c = 0;           /* the running counter */
+    int64_t d = frame_len;   /* offset into the open frame; frame_len: none */
+    int64_t f = 0;           /* the open frame's anchor */
+    int64_t last_marker = -1;
+    for (int64_t p = 0; p < len; ++p) {
+      int64_t v[3];
+      if (ids[first + p] == image_token_id) { /* a new frame */
+        f = c;
+        c = f + s + 1;
+        d = 0;
+        last_marker = p;
+      }
+      if (d < frame_len) {
+        if (d == 0) {                /* <image> */
+          v[0] = f;
+          v[1] = v[2] = f - 1;
+        } else if (d <= s * s) {     /* image row k */
+          const int64_t k = d - 1;
+          v[0] = f;
+          v[1] = f + k / s;
+          v[2] = f + k % s;
+        } else if (d == s * s + 1) { /* </image> */
+          v[0] = f;
+          v[1] = v[2] = f + s;
+        } else {                     /* the "\n" */
+          v[0] = v[1] = v[2] = f;
+        }
+        ++d;
+      } else {                       /* text */
+        v[0] = v[1] = v[2] = c;
+        ++c;
+      }
+      for (int r = 0; r < 3; ++r) pos[r * n_tokens + first + p] = (int32_t)v[r];
+    }
+    if (last_marker < 0) {
+      start_out[b] = TEXT_ONLY_START;
+      amount_out[b] = 0;
+    } else {
+      /* the counter after the last frame is that frame's anchor + s + 1, and
+       * the text at index start takes it */
+      const int64_t start = last_marker + frame_len;
+      const int64_t last_anchor_next = f + s + 1;
+      start_out[b] = (int32_t)start;
+      amount_out[b] = (int32_t)(start - last_anchor_next);
+    }
+  }
+  return ORC_OK;
+}
+
 /* Decode / continuation: the token at absolute index p = cache_len[b] of
  * sequence b, with that sequence's start and amount.  Generated tokens sit at
  * p - amount on all three planes ([P1]; [P2]'s canvas table counts generated

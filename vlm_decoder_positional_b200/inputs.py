@@ -78,12 +78,14 @@ def text_ids(rng: np.random.Generator, n: int, avoid=(IMAGE_TOKEN_ID,)) -> np.nd
     return ids.astype(np.int32)
 
 
-def frame_ids(row_ids: str = "v_plus_k") -> np.ndarray:
-    """The 67 ids of one image frame: <image>, 64 rows, </image>, "\\n"."""
+def frame_ids(row_ids: str = "v_plus_k", grid_side: int = 8) -> np.ndarray:
+    """The ids of one image frame: <image>, grid_side^2 rows, </image>, "\\n"
+    (67 ids for the 448x448 thumbnail's 8x8 grid)."""
+    n_rows = grid_side * grid_side
     if row_ids == "v_plus_k":
-        rows = VOCAB + np.arange(ROWS_PER_IMAGE)
+        rows = VOCAB + np.arange(n_rows)
     elif row_ids == "pad":
-        rows = np.full(ROWS_PER_IMAGE, IMAGE_PAD_ID)
+        rows = np.full(n_rows, IMAGE_PAD_ID)
     else:
         raise ValueError(row_ids)
     return np.concatenate([[IMAGE_TOKEN_ID], rows, [IMAGE_END_ID, NEWLINE_ID]]).astype(np.int32)
@@ -99,6 +101,32 @@ def prompt_ids(rng: np.random.Generator, length: int, origin: int,
         if origin < length:
             ids[origin:end] = fr[: end - origin]
     return ids
+
+
+def prompt_ids_frames(rng: np.random.Generator, length: int, origins: Sequence[int],
+                      grid_side: int = 8) -> np.ndarray:
+    """One prompt of ``length`` ids with a frame of grid_side^2 rows starting at
+    each of ``origins`` (laid in order, each truncated by the end of the prompt
+    and overwritten from the next origin on if they overlap)."""
+    ids = text_ids(rng, length)
+    fr = frame_ids("v_plus_k", grid_side)
+    for o in sorted(origins):
+        if 0 <= o < length:
+            end = min(length, o + fr.shape[0])
+            ids[o:end] = fr[: end - o]
+    return ids
+
+
+def spaced_origins(rng: np.random.Generator, count: int, lo: int, hi: int,
+                   gap: int) -> list:
+    """``count`` sorted origins in [lo, hi] at least ``gap`` apart (uniform
+    over such sets: draw count points in [lo, hi - (count-1) gap], sort,
+    spread)."""
+    span = hi - (count - 1) * gap
+    if span < lo:
+        raise ValueError("no room for that many spaced origins")
+    base = np.sort(rng.integers(lo, span + 1, size=count))
+    return [int(b + i * gap) for i, b in enumerate(base)]
 
 
 def pack(prompts: Sequence[np.ndarray]):
