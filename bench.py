@@ -1,17 +1,22 @@
 """Benchmark of the canvas M-RoPE hot path on B200.
 
-One step = the whole path over one batch: cmr_positions (planes from ids) then
-cmr_rotate_qk (fused cos/sin + rotate of Q and K, every layer), on the
-6-layer workload: 32 prompts x 8192 tokens with one image frame each, Q [6,
-262144, 8, 256] and K [6, 262144, 2, 256] bf16, rot_dim 64, theta 1e7,
-sections [11, 11, 10].  The rotate kernel touches 4.03 GB per step, far more
-than the 126 MB L2, so no L2 flush is needed between steps.
+One step = the whole path over one batch: the planes from the ids, then the
+fused cos/sin + rotate of Q and K (every layer), through the one-call entry
+point cmr_positions_rotate_qk (the rotation launched to overlap the positions
+kernels), on the 6-layer workload: 32 prompts x 8192 tokens with one image
+frame each, Q [6, 262144, 8, 256] and K [6, 262144, 2, 256] bf16, rot_dim 64,
+theta 1e7, sections [11, 11, 10].  The rotate kernel touches 4.03 GB per step,
+far more than the 126 MB L2, so no L2 flush is needed between steps.
+--step separate calls cmr_positions and cmr_rotate_qk one after the other
+instead, and times the rotate launch on its own.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...   (weak scaling: one batch per GPU)
+    python bench.py --probe copy-pattern   (the staged copy-pattern ceiling alone)
 
-Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle
-(single thread) on a bounded sample of the same workload.
+Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle on
+all host cores (a thread pool over token ranges) on a bounded sample of the
+same workload.
 """
 import argparse
 import datetime
@@ -36,6 +41,7 @@ from vlm_decoder_positional_b200 import cmr, inputs, pipeline, shard  # noqa: E4
 METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/K, 1 GPU"
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (DGX figure)
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_staged.cu",
                   "vlm_decoder_positional_b200/csrc/tma.cuh",
@@ -69,6 +75,23 @@ def workload_label(wl):
             f"{wl.num_layers} layers, Q [{wl.num_layers},{t},{wl.hq},{wl.head_dim}] "
             f"K [{wl.num_layers},{t},{wl.hk},{wl.head_dim}] bf16, rot_dim "
             f"{wl.rot_dim}, theta {wl.theta:g}, sections {list(wl.sections)}")
+
+
+def config_dict(args, wl, tokens_all, world, rot_b):
+    """The workload's config, the same for both arms of the benchmark."""
+    return {"workload": workload_label(wl), "global_batch": tokens_all,
+            "launch": args.launch, "op": args.op, "step": step_kind(args, wl),
+            "seq_len": wl.n_tokens // max(wl.num_seqs, 1),
+            "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'whole prompts split over ranks'}, no data-path collective)",
+            "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
+                  " no flush" % (rot_b / 1e9)}
+
+
+def step_kind(args, wl):
+    """'one-call' when a prefill step runs the positions + rotate entry point."""
+    if args.op == "rotate" and wl.cache_len is None and args.step == "fused":
+        return "one-call"
+    return "separate"
 
 
 def measured_peak():
@@ -290,6 +313,9 @@ def run_reference(args):
         return 0
     # the same prompts (ids); Q/K drawn only for the sampled tokens
     wl = inputs.make_config(args.workload, device="cpu", with_qk=False)
+    if args.layers is not None:
+        wl.num_layers = args.layers
+    full_tokens = wl.num_seqs if wl.cache_len is not None else wl.n_tokens
     cores = host_cores()
     per_step = max(1.0, args.reference_budget_s / (args.steps + args.warmup))
     n_max = min(wl.num_seqs if wl.cache_len is not None else wl.n_tokens, 200_000)
@@ -310,11 +336,14 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-        "config": {"workload": workload_label(wl), "global_batch": wl.n_tokens,
-                   "seq_len": wl.n_tokens // wl.num_seqs,
-                   "parallelism": f"cpu oracle, {cores} threads"},
+        "config": config_dict(args, wl, full_tokens * args.gpus if args.scaling == "weak"
+                              else full_tokens, args.gpus,
+                              rotate_bytes(full_tokens, wl.num_layers, wl.hq, wl.hk,
+                                           wl.rot_dim) if args.op != "cache" else
+                              cache_bytes(full_tokens, wl.num_layers, wl.hq, wl.hk, wl.rot_dim,
+                                          wl.head_dim)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample + f", the fp64 oracle on {cores} host threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }), flush=True)
@@ -400,6 +429,10 @@ def run_ours(args):
         else:
             plan = [("rotate", lambda: cmr.rotate_qk_shift(wl.q, wl.k, start, amount,
                                                            pos_offset=cache_len, **rope))]
+    elif step_kind(args, wl) == "one-call":
+        plan = [("rotate", lambda: cmr.positions_rotate_qk(
+            ids, cu, wl.q, wl.k, wl.theta, wl.sections, wl.rot_dim, wl.image_token_id,
+            out=(pos, start, amount)))]
     else:
         plan = [("positions", lambda: cmr.positions(ids, cu, wl.image_token_id,
                                                     out=(pos, start, amount)))]
@@ -414,7 +447,9 @@ def run_ours(args):
                 wl.q, wl.k, v, start, amount, k_cache, v_cache, cu_seqlens=cu, **rope)))
     calls = dict(plan)
     if args.launch == "graph":
-        # one CUDA graph per call, each holding its single kernel launch
+        # one CUDA graph per call: a rotate form's single kernel, or the
+        # positions form's memset and two kernels (the one-call step also holds
+        # the rotation, behind a programmatic edge)
         for fn in calls.values():
             fn()
         torch.cuda.synchronize(dev)
@@ -440,6 +475,9 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    # the rotate kernel the library actually launched (recorded at the launch
+    # or at its capture into the graph)
+    kernel_ran = cmr.last_rotate_kernel() or kernel
 
     rot_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                   for _ in range(args.steps)]
@@ -462,7 +500,12 @@ def run_ours(args):
     ms_max = shard.max_over_ranks(ms, dist, dev)
     # tokens processed by all ranks in one step
     tokens_all = tokens_per_step * world if args.scaling == "weak" else global_tokens
-    launches = args.steps * len(plan)
+    # kernels per step: the positions form launches two (origin scan, planes),
+    # each rotate form one
+    per_step = {"positions": 2, "rotate": 1}
+    launches = args.steps * sum(per_step[name] for name, _ in plan)
+    if step_kind(args, wl) == "one-call":
+        launches = args.steps * 3
 
     # end to end through the public API from pinned host memory
     if args.op == "rotate":
@@ -471,15 +514,36 @@ def run_ours(args):
         e2e = {"skipped": f"--op {args.op} times the device step only; the end-to-end path "
                           "is measured with --op rotate"}
 
+    ceiling = None
+    if args.op == "rotate" and kernel_ran == "rotate_qk_staged_kernel":
+        ceiling = run_copy_pattern_probe(wl, dev, stream)
+
     if rank == 0:
         peak, peak_src = measured_peak()
         rot_avg_s = statistics.mean(rot_ms) / 1e3
         achieved = rot_b / rot_avg_s / 1e9
-        traffic = recorded_traffic(wl.name, kernel) if args.op == "rotate" else None
+        traffic = recorded_traffic(wl.name, kernel_ran) if args.op == "rotate" else None
         value = tokens_all * args.steps / (ms_max / 1e3)
+        one_call = step_kind(args, wl) == "one-call"
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = run_cpu_baseline(wl, args.cpu_seconds)
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "kernel": kernel_ran,
+                    "algorithmic_bytes_per_launch": rot_b,
+                    "avg_launch_ms": rot_avg_s * 1e3,
+                    "timed": ("the whole one-call step (CUDA events around it): the positions "
+                              "kernels and the rotation overlapping them, an upper bound of the "
+                              "rotate kernel's own duration" if one_call else
+                              "the rotate launch alone (CUDA events around it)"),
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                    if peak_src == "measured" else "fallback 6650 GB/s",
+                    "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS}
+        if ceiling is not None:
+            roofline["ceiling"] = ceiling["gbs"]
+            roofline["frac_of_ceiling"] = achieved / ceiling["gbs"]
+            roofline["ceiling_source"] = ceiling["what"]
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -487,25 +551,188 @@ def run_ours(args):
             "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 Q/K, uniform text ids, one 448x448 frame "
                     "per prompt)",
-            "config": {"workload": workload_label(wl), "global_batch": tokens_all,
-                       "launch": args.launch, "op": args.op,
-                       "seq_len": n // max(b, 1),
-                       "parallelism": f"dp{world} ({'independent batches' if args.scaling == 'weak' else 'whole prompts split over ranks'}, no data-path collective)",
-                       "l2": "inputs larger than L2 (rotate touches %.2f GB per step, L2 126 MB);"
-                             " no flush" % (rot_b / 1e9)},
+            "config": config_dict(args, wl, tokens_all, world, rot_b),
             "hbm_gbs": achieved, "pct_of_peak": 100.0 * achieved / peak,
+            "pct_of_spec_peak": 100.0 * achieved / SPEC_HBM_GBS,
             "token_layers_per_s": value * L,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "kernel": kernel,
-                         "algorithmic_bytes_per_launch": rot_b,
-                         "avg_launch_ms": rot_avg_s * 1e3,
-                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
-                         if peak_src == "measured" else "fallback 6650 GB/s"},
+            "roofline": roofline,
             "positions_bytes_per_step": positions_bytes(n, b),
-            "positions_avg_ms": statistics.mean(pos_ms),
+            "positions_avg_ms": None if one_call else statistics.mean(pos_ms),
             "e2e": e2e, "gpu_launches": launches, "clocks": clocks.summary(),
             "cpu_baseline": cpu, "impl": "ours",
+        }
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def probe_lib():
+    import ctypes
+    from vlm_decoder_positional_b200 import build as libbuild
+    libbuild.build()
+    lib = ctypes.CDLL(libbuild.PROBE_LIB)
+    f = lib.cmr_probe_copy_pattern
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                  ctypes.c_void_p]
+    return f
+
+
+def run_copy_pattern_probe(wl, dev, stream, launches=10, warmup=3):
+    """The ceiling of the staged rotation's access pattern: copy_pattern_kernel
+    moves the same rotated dims of Q and K through the same TMA staging with no
+    math (an identity copy), timed like the rotate launch (CUDA events around
+    each of `launches` launches).  Returns GB/s over the Q/K bytes it moves."""
+    f = probe_lib()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = wl.q.shape[1]
+    args = (wl.q.data_ptr(), wl.k.data_ptr(), n, wl.num_layers, wl.hq, wl.hk, wl.head_dim,
+            status.data_ptr(), stream.cuda_stream)
+    for _ in range(warmup):
+        if f(*args) != 0:
+            raise RuntimeError("copy-pattern probe: launch refused")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(launches)]
+    torch.cuda.synchronize(dev)
+    for a, z in ev:
+        a.record(stream)
+        f(*args)
+        z.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError("copy-pattern probe: a bounded wait gave up")
+    ms = statistics.mean(a.elapsed_time(z) for a, z in ev)
+    moved = n * wl.num_layers * (wl.hq + wl.hk) * 64 * 2 * 2
+    return {"gbs": moved / (ms / 1e3) / 1e9, "ms": ms, "bytes": moved,
+            "what": "copy_pattern_kernel (libcmr_probe.so): the staged rotation's TMA boxes "
+                    "loaded and stored back unchanged, no math; mean of %d launches" % launches}
+
+
+def run_probe_only(args):
+    """--probe copy-pattern: the ceiling probe alone on the workload's Q/K."""
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    wl = inputs.make_config(args.workload, device=dev)
+    res = run_copy_pattern_probe(wl, dev, torch.cuda.current_stream(dev), launches=args.steps,
+                                 warmup=args.warmup)
+    peak, src = measured_peak()
+    print(json.dumps({"probe": "copy-pattern", "workload": workload_label(wl),
+                      "gbs": res["gbs"], "ms_per_launch": res["ms"], "bytes": res["bytes"],
+                      "peak": peak, "peak_source": src, "frac_of_peak": res["gbs"] / peak,
+                      "launches": args.steps, "what": res["what"]}), flush=True)
+    return 0
+
+
+def run_frames(args):
+    """--op frames: one step = cmr_positions_frames (multi-frame canvas planes)
+    on the multi-frame workload (256 prompts x 65,536 tokens, 32 frames each,
+    grid side --grid-side), graph-replayed, CUDA events around each call."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    cmr.lib()
+    seed = shard.rank_seed(inputs.BASE_SEED + 6, rank)
+    wl = inputs.make_frames_workload(frames=args.frames_per_prompt, grid_side=args.grid_side,
+                                     seed=seed)
+    n, b = wl.n_tokens, wl.num_seqs
+    ids = torch.from_numpy(wl.ids).to(dev)
+    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+    pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+    start = torch.empty(b, dtype=torch.int32, device=dev)
+    amount = torch.empty(b, dtype=torch.int32, device=dev)
+    ws = torch.empty(cmr.positions_frames_workspace_bytes(b, n), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        cmr.positions_frames(ids, cu, args.grid_side, out=(pos, start, amount), workspace=ws)
+
+    call()
+    torch.cuda.synchronize(dev)
+    if args.launch == "graph":
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call()
+        call = g.replay
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        t_begin.record(stream)
+        for a, z in ev:
+            a.record(stream)
+            call()
+            z.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    ms_max = shard.max_over_ranks(t_begin.elapsed_time(t_end), dist, dev)
+    call_ms = statistics.mean(a.elapsed_time(z) for a, z in ev)
+    moved = positions_bytes(n, b)
+    if rank == 0:
+        peak, peak_src = measured_peak()
+        achieved = moved / (call_ms / 1e3) / 1e9
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cores = 1
+            take = 1
+            t0 = time.perf_counter()
+            while True:  # whole prompts, about --cpu-seconds of oracle work
+                oracle.positions_frames(wl.ids[: wl.cu_seqlens[take]], wl.cu_seqlens[: take + 1],
+                                        wl.image_token_id, args.grid_side)
+                dt = time.perf_counter() - t0
+                if dt > args.cpu_seconds or take == b:
+                    break
+                take = min(b, take * 2)
+                t0 = time.perf_counter()
+            cpu = {"value": int(wl.cu_seqlens[take]) / dt, "unit": UNIT, "cores": cores,
+                   "kind": "oracle",
+                   "sample": f"multi-frame planes of the first {take} prompts "
+                             f"({int(wl.cu_seqlens[take])} tokens), 1 thread, {dt:.2f} s"}
+        tokens_all = n * world
+        out = {
+            "metric": METRIC, "value": tokens_all * args.steps / (ms_max / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int32",
+            "data": "synthetic (seeded uniform text ids, frames on a grid_side x grid_side grid)",
+            "config": {"workload": f"{wl.name}: {b} prompts x {n // b} tokens, "
+                                   f"{args.frames_per_prompt} frames each, grid side "
+                                   f"{args.grid_side}", "global_batch": tokens_all,
+                       "launch": args.launch, "op": "frames", "step": "separate",
+                       "seq_len": n // b, "parallelism": f"dp{world} (independent batches, no "
+                                                         "data-path collective)",
+                       "l2": "inputs larger than L2 (%.0f MB of ids and planes per step, L2 "
+                             "126 MB); no flush" % (moved / 1e6)},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "frames_positions_kernel (+ frames_summary_kernel)",
+                         "algorithmic_bytes_per_launch": moved, "avg_launch_ms": call_ms,
+                         "timed": "the whole call (CUDA events around it): the summary and "
+                                  "planes kernels",
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_src == "measured" else "fallback 6650 GB/s",
+                         "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS},
+            "e2e": {"skipped": "--op frames times the device step only"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "cpu_baseline": cpu,
+            "impl": "ours",
         }
         print(json.dumps(out), flush=True)
     if dist:
@@ -595,7 +822,7 @@ def run_e2e(args, wl, dev, stream, dist, tokens_all):
             "path": ("pinned host -> rotated dims in (pitched copies), cmr.rotate_qk_shift, "
                      "rotated dims out -> pinned host" if decode else
                      "pinned host -> HostPipeline: chunks of whole prompts, rotated dims in "
-                     "(pitched copies), cmr.positions + cmr.rotate_qk, rotated dims out, on "
+                     "(pitched copies), cmr.positions_rotate_qk, rotated dims out, on "
                      "three streams -> pinned host")}
 
 
@@ -611,9 +838,20 @@ def main():
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: a full batch per GPU (default); strong: one batch split by "
                          "whole prompts")
-    ap.add_argument("--op", choices=["rotate", "shift", "cache"], default="rotate",
+    ap.add_argument("--op", choices=["rotate", "shift", "cache", "frames"], default="rotate",
                     help="rotate: planes from pos (default); shift: planes derived in the "
-                         "rotate kernel; cache: rotate + KV-cache write")
+                         "rotate kernel; cache: rotate + KV-cache write; frames: the "
+                         "multi-frame planes alone on their own workload")
+    ap.add_argument("--grid-side", type=int, default=8,
+                    help="--op frames: side of each frame's grid (8: 448x448 thumbnail)")
+    ap.add_argument("--frames-per-prompt", type=int, default=32,
+                    help="--op frames: frames in each of the 256 x 65,536-token prompts")
+    ap.add_argument("--step", choices=["fused", "separate"], default="fused",
+                    help="fused: a prefill rotate step is one cmr_positions_rotate_qk call "
+                         "(default); separate: cmr_positions then cmr_rotate_qk, the rotate "
+                         "launch timed on its own")
+    ap.add_argument("--probe", choices=["copy-pattern"], default=None,
+                    help="run only the copy-pattern ceiling probe (--steps launches)")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="graph: replay a captured CUDA graph per call (default); eager: "
                          "launch through the Python binding every step")
@@ -627,6 +865,10 @@ def main():
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.probe:
+        return run_probe_only(args)
+    if args.op == "frames":
+        return run_frames(args)
     return run_ours(args)
 
 

@@ -29,6 +29,7 @@
 #ifndef CMR_H_
 #define CMR_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -54,8 +55,10 @@ typedef enum cmr_status {
 /* Bits a kernel ORs into the optional device status word. */
 #define CMR_DEVICE_BAD_CU_SEQLENS 1 /* cu_seqlens not 0 .. n_tokens, non-decreasing */
 #define CMR_DEVICE_CACHE_RANGE 2    /* a token's cache index or slot outside the cache */
-#define CMR_DEVICE_WAIT_TIMEOUT 4   /* a staged kernel waited over 1 s for a copy and gave
-                                       up; rows of the tiles involved may be unrotated */
+#define CMR_DEVICE_WAIT_TIMEOUT 4   /* a staged kernel waited over 1 s for one of its own
+                                       copies and gave up: the call's results are not to be
+                                       trusted (rows of the tiles involved may be unrotated
+                                       or half written) */
 
 /* Position rules for cmr_positions_chunk. */
 #define CMR_RULE_CANVAS 0    /* this model's canvas rule: start = O + 67, amount 58 */
@@ -87,9 +90,15 @@ typedef enum cmr_status {
  *   out_pos      device int32 [3, n_tokens], plane-major: T row, H row, W row
  *   out_start, out_amount   device int32 [num_seqs]
  *   device_status  optional device int32 [1] (may be NULL).  If cu_seqlens is
- *                malformed, the kernel ORs CMR_DEVICE_BAD_CU_SEQLENS into it
- *                and writes nothing for the prompts whose bounds are invalid.
+ *                malformed, the kernels OR CMR_DEVICE_BAD_CU_SEQLENS into it
+ *                and write no planes for the prompts whose bounds are invalid
+ *                (their out_start / out_amount entries are then unspecified).
  *                The library never clears it.
+ * The work is a memset of out_start and two kernels: a scan of each slice of
+ * each prompt for its first marker, which lowers out_start[b] with an atomic
+ * min (every id is read once), then the planes and the state.  out_start is
+ * therefore written during the call; it must not be read or written by other
+ * work in flight.
  * Errors: CMR_EINVAL for null required pointers, negative sizes, num_seqs = 0
  * with n_tokens > 0, or n_tokens > INT32_MAX. */
 CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
@@ -138,6 +147,51 @@ CMR_API cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seq
                                        const int32_t* in_amount, int32_t* out_pos,
                                        int32_t* out_start, int32_t* out_amount,
                                        int32_t* device_status, cmr_stream_t stream);
+
+/* Planes of prompts holding several image frames, on an s x s grid of any
+ * side (s = grid_side: 8 for the 448x448 thumbnail's 64 rows, 16 for a grid
+ * of 256).  The pages print the canvas for one thumbnail only (HF card
+ * mlboydaisuke/MiniCPM-V-4.7-1B-CoreAI, "How the VLM rides the text-only
+ * engine"); the MNN card ("Validation") says sliced and multi-image prompts
+ * were checked too, without values.  The reading implemented: a running
+ * counter c gives each text token (c, c, c) and advances by 1; EVERY marker
+ * opens a frame of s*s + 3 tokens anchored at the counter's value f:
+ *   <image> (f, f-1, f-1); row k < s*s (f, f + k/s, f + k%s) (row-major);
+ *   </image> (f, f+s, f+s); the "\n" after it (f, f, f);
+ * and the counter then stands at f + s + 1, one past the frame's largest
+ * coordinate (the card's 9 = max(H, W) + 1), also when the next marker or the
+ * end of the prompt cuts the frame short.  With one marker and s = 8 this is
+ * cmr_positions.  The state is start = (last marker) + s*s + 3 and amount with
+ * every later text token at p - amount, so cmr_positions_step and the shift
+ * forms continue a prompt after its last frame; text-only (2^30, 0).
+ *
+ *   ids, cu_seqlens, num_seqs, n_tokens, image_token_id, out_pos, out_start,
+ *   out_amount, device_status   as in cmr_positions
+ *   grid_side      1 .. 128
+ *   workspace      device memory, 16-byte aligned, of workspace_bytes >= 16 *
+ *                  num_seqs; cmr_positions_frames_workspace_bytes gives the
+ *                  size for full parallelism (16 B per sequence per slice of
+ *                  about 2,048 tokens); a smaller one works with fewer,
+ *                  longer slices.  It holds one summary per slice between the
+ *                  call's two kernels; its contents before and after a call
+ *                  do not matter, but calls that overlap on the device must
+ *                  not share it.
+ * Every coordinate must fit in int32.  Two kernels: a per-slice summary (marker
+ * count, first and last marker, text between frames), then the planes, the
+ * second launched to overlap the first.
+ * Errors: as cmr_positions, plus CMR_EINVAL for grid_side outside 1 .. 128 and a
+ * missing, misaligned or too small workspace. */
+CMR_API cmr_status cmr_positions_frames(const int32_t* ids, const int32_t* cu_seqlens,
+                                        int32_t num_seqs, int64_t n_tokens,
+                                        int32_t image_token_id, int32_t grid_side,
+                                        int32_t* out_pos, int32_t* out_start,
+                                        int32_t* out_amount, void* workspace,
+                                        size_t workspace_bytes, int32_t* device_status,
+                                        cmr_stream_t stream);
+
+/* Workspace bytes for cmr_positions_frames at full parallelism (0 for no
+ * sequences).  No CUDA call is made. */
+CMR_API size_t cmr_positions_frames_workspace_bytes(int32_t num_seqs, int64_t n_tokens);
 
 /* Planes of one new token per sequence, for decode and continuation (port
  * notes: generated tokens sit at p - amount; the canvas table's last row,
@@ -192,6 +246,30 @@ CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n
                          const int32_t sections[3], int32_t rot_dim,
                          int32_t* device_status, cmr_stream_t stream);
 
+/* The whole path in one call: cmr_positions, then cmr_rotate_qk with the
+ * planes just written (same arguments, same results, bit for bit).  The
+ * rotation is launched with programmatic stream serialization behind the
+ * positions kernels: its CTAs start while the planes are being written, the
+ * TMA loads of Q and K (which the positions kernels never touch) go out at
+ * once, and only the rotation itself waits for the planes.  Launching the
+ * two separately cannot overlap them, because a caller's kernel before a
+ * plain cmr_rotate_qk may still be writing Q/K when it signals.
+ *
+ *   ids, cu_seqlens, num_seqs, n_tokens, image_token_id, out_pos, out_start,
+ *   out_amount     as in cmr_positions (out_pos is also the rotation's pos)
+ *   q, k, num_layers, hq, hk, head_dim, theta, sections, rot_dim
+ *                  as in cmr_rotate_qk (n_tokens tokens)
+ *   device_status  optional, receives the bits of both steps
+ * Errors: every check of both calls runs before anything is enqueued. */
+CMR_API cmr_status cmr_positions_rotate_qk(const int32_t* ids, const int32_t* cu_seqlens,
+                                           int32_t num_seqs, int64_t n_tokens,
+                                           int32_t image_token_id, int32_t* out_pos,
+                                           int32_t* out_start, int32_t* out_amount, void* q,
+                                           void* k, int32_t num_layers, int32_t hq, int32_t hk,
+                                           int32_t head_dim, double theta,
+                                           const int32_t sections[3], int32_t rot_dim,
+                                           int32_t* device_status, cmr_stream_t stream);
+
 /* cmr_rotate_qk with the planes derived inside the kernel instead of read
  * from pos [3, n_tokens]: token t of prompt b (cu[b] <= t < cu[b+1]) sits at
  * absolute index p = pos_offset[b] + t - cu[b] and gets the canvas table's
@@ -217,12 +295,18 @@ CMR_API cmr_status cmr_rotate_qk_shift(void* q, void* k, const int32_t* cu_seqle
                                        const int32_t sections[3], int32_t rot_dim,
                                        int32_t* device_status, cmr_stream_t stream);
 
-/* Name of the kernel that cmr_rotate_qk / cmr_rotate_qk_shift launch for these
- * shapes: "rotate_qk_staged_kernel" (TMA-staged, rot_dim 64, large batches) or
- * "rotate_qk_kernel" (register-resident rows, every other case).  The staged
- * kernel also needs the driver to encode tensor maps for the buffers (any
- * driver for sm_100a does, for contiguous Q/K of under 1 TB per layer);
- * otherwise the call takes rotate_qk_kernel.
+/* Name of the kernel that cmr_rotate_qk / cmr_rotate_qk_shift /
+ * cmr_positions_rotate_qk launch for these shapes: "rotate_qk_staged_kernel"
+ * (TMA-staged, rot_dim 64, large batches) or "rotate_qk_kernel"
+ * (register-resident rows, every other case).  It is a prediction from the
+ * shapes alone; a call still takes rotate_qk_kernel when
+ *   - the driver cannot encode tensor maps for the buffers (any driver for
+ *     sm_100a can, for contiguous 16-byte aligned Q/K of under 1 TB per layer);
+ *   - the staged ring needs more than 48 KB of shared memory (more than 24
+ *     head rows of Q and K per token: not this model's 8 + 2), the process has
+ *     not launched that form on this device before, and the call is being
+ *     captured into a CUDA graph (or its stream cannot be queried).
+ * cmr_last_rotate_kernel names the kernel a call actually launched.
  * Returns NULL when the shapes are invalid or there is nothing to launch.
  * Static strings; no CUDA call is made. */
 CMR_API const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, int32_t hq,
@@ -230,10 +314,13 @@ CMR_API const char* cmr_rotate_qk_kernel(int64_t n_tokens, int32_t num_layers, i
 
 /* The same for cmr_rotate_qk_cache: "rotate_qk_cache_staged_kernel" (TMA-staged,
  * rot_dim 64, large batches, head_dim <= 256, K/V token rows a multiple of
- * 128 B) or "rotate_qk_cache_kernel".  The staged kernel's first launch in a
- * process needs more than the default shared memory; if that first launch is
- * being captured into a CUDA graph, it takes rotate_qk_cache_kernel.  NULL when
- * the shapes are invalid or there is nothing to launch. */
+ * 128 B) or "rotate_qk_cache_kernel".  A call still takes
+ * rotate_qk_cache_kernel when the driver cannot encode tensor maps for the
+ * buffers, or when the staged kernel's ring needs more than 48 KB of shared
+ * memory (this model's 8 + 2 heads: 73 KB), the process has not launched it
+ * on this device before, and the call is being captured into a CUDA graph (or
+ * its stream cannot be queried).  NULL when the shapes are invalid or there is
+ * nothing to launch. */
 CMR_API const char* cmr_rotate_qk_cache_kernel(int64_t n_tokens, int32_t num_layers,
                                                int32_t hq, int32_t hk, int32_t head_dim,
                                                int32_t rot_dim);
@@ -298,6 +385,12 @@ CMR_API const char* cmr_status_string(cmr_status s);
 
 /* One-line reason for the last non-CMR_OK return on the calling thread. */
 CMR_API const char* cmr_last_error_message(void);
+
+/* Name of the rotate kernel that the calling thread's last successful rotate
+ * call enqueued ("rotate_qk_staged_kernel", "rotate_qk_kernel",
+ * "rotate_qk_cache_staged_kernel" or "rotate_qk_cache_kernel"); "" before the
+ * first.  Static strings; no CUDA call is made. */
+CMR_API const char* cmr_last_rotate_kernel(void);
 
 /* ABI version: major * 10000 + minor * 100 + patch. */
 CMR_API int32_t cmr_version(void);

@@ -28,10 +28,12 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
-                          "cmr_rotate_qk", "cmr_rotate_qk_shift", "cmr_rotate_qk_cache", "cmr_rotate_qk_kernel",
-                          "cmr_rotate_qk_cache_kernel",
-                          "cmr_copy_rotated_dims", "cmr_status_string",
-                          "cmr_last_error_message", "cmr_version"}
+                          "cmr_rotate_qk", "cmr_positions_rotate_qk", "cmr_rotate_qk_shift",
+                          "cmr_rotate_qk_cache", "cmr_rotate_qk_kernel",
+                          "cmr_rotate_qk_cache_kernel", "cmr_copy_rotated_dims",
+                          "cmr_status_string", "cmr_last_error_message",
+                          "cmr_last_rotate_kernel", "cmr_version", "cmr_positions_frames",
+                          "cmr_positions_frames_workspace_bytes"}
     assert set(names) == set(cmr.SIGNATURES)
 
 
@@ -50,7 +52,8 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 20000
+    assert lib.cmr_version() == 20100
+    assert lib.cmr_last_rotate_kernel() == b""  # nothing launched on this thread
 
 
 SEC = (ctypes.c_int32 * 3)(11, 11, 10)
@@ -99,6 +102,57 @@ def test_positions_empty_batch_is_a_no_op(lib):
     assert lib.cmr_positions(None, None, 0, 0, 248078, None, None, None, None, None) == 0
     assert lib.cmr_positions_step(None, None, None, 0, None, None) == 0
     assert lib.cmr_positions_step(None, None, None, -1, None, None) == cmr.CMR_EINVAL
+
+
+@pytest.mark.parametrize("kw", [
+    dict(theta=0.0), dict(rot_dim=24), dict(sections=(12, 11, 10)), dict(hq=0, hk=0),
+    dict(num_seqs=-1), dict(num_seqs=0, n_tokens=10), dict(cu=None), dict(q=FAKE + 2),
+])
+def test_positions_rotate_rejects_bad_arguments_of_either_step(lib, kw):
+    # the checks of both steps run before anything is enqueued; with no tokens
+    # the rotation's own arguments are still checked
+    a = dict(ids=None, cu=None, num_seqs=0, n_tokens=0, q=None, k=None, hq=8, hk=2,
+             theta=1e7, sections=(11, 11, 10), rot_dim=64)
+    if "cu" in kw or "q" in kw:
+        a.update(ids=FAKE, cu=FAKE, num_seqs=1, n_tokens=10, q=FAKE, k=FAKE)
+    a.update(kw)
+    sec = (ctypes.c_int32 * 3)(*a["sections"])
+    st = lib.cmr_positions_rotate_qk(a["ids"], a["cu"], a["num_seqs"], a["n_tokens"], 248078,
+                                     FAKE, FAKE, FAKE, a["q"], a["k"], 1, a["hq"], a["hk"], 256,
+                                     a["theta"], sec, a["rot_dim"], None, None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+
+
+@pytest.mark.parametrize("kw", [
+    dict(grid_side=0), dict(grid_side=129), dict(ws=None), dict(ws_bytes=16 * 3 - 1),
+    dict(ws=FAKE + 8), dict(num_seqs=-1), dict(cu=None),
+])
+def test_positions_frames_rejects_bad_arguments_on_the_host(lib, kw):
+    a = dict(ids=FAKE, cu=FAKE, num_seqs=3, n_tokens=30, grid_side=8, ws=FAKE, ws_bytes=1 << 20)
+    a.update(kw)
+    st = lib.cmr_positions_frames(a["ids"], a["cu"], a["num_seqs"], a["n_tokens"], 248078,
+                                  a["grid_side"], FAKE, FAKE, FAKE, a["ws"], a["ws_bytes"], None,
+                                  None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
+
+
+def test_positions_frames_workspace_size():
+    # 16 bytes per sequence per slice of about 2,048 tokens
+    assert cmr.positions_frames_workspace_bytes(0, 0) == 0
+    assert cmr.positions_frames_workspace_bytes(1, 80) == 16
+    assert cmr.positions_frames_workspace_bytes(32, 32 * 8192) == 16 * 32 * 4
+    assert cmr.positions_frames_workspace_bytes(1, 300_000) == 16 * 147
+    assert lib_ok(cmr.lib().cmr_positions_frames(None, None, 0, 0, 248078, 8, None, None, None,
+                                                 None, 0, None, None))
+
+
+def lib_ok(status):
+    return status == cmr.CMR_OK
+
+
+def test_positions_rotate_of_nothing_is_a_no_op(lib):
+    assert lib.cmr_positions_rotate_qk(None, None, 0, 0, 248078, None, None, None, None, None, 1,
+                                       8, 2, 256, 1e7, SEC, 64, None, None) == 0
 
 
 @pytest.mark.parametrize("kw", [

@@ -64,3 +64,8 @@ def test_reference_arm_prints_one_json_line():
     assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    # the same config keys (and workload) as the GPU arm's line
+    assert set(d["config"]) == {"workload", "global_batch", "launch", "op", "step", "seq_len",
+                                "parallelism", "l2"}
+    assert d["config"]["workload"].startswith("c1_single_prompt_80: 1 prompts x 80 tokens")
+    assert d["config"]["global_batch"] == 80

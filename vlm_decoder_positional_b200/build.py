@@ -1,9 +1,11 @@
-"""Builds libcmr.so, the C-ABI library, in-tree with nvcc for sm_100a (B200).
+"""Builds libcmr.so, the C-ABI library, in-tree with nvcc for sm_100a (B200),
+and libcmr_probe.so, the benchmark's copy-pattern ceiling probe.
 
     python -m vlm_decoder_positional_b200.build [--force] [--verbose-ptxas]
 
-The CUDA runtime is linked statically, so the library needs only the NVIDIA
-driver at run time.  Only the symbols declared in include/cmr.h are exported.
+The CUDA runtime is linked statically, so the libraries need only the NVIDIA
+driver at run time.  Only the symbols declared in include/cmr.h are exported
+from libcmr.so.
 """
 import argparse
 import glob
@@ -15,6 +17,8 @@ ROOT = os.path.dirname(PKG)
 INCLUDE = os.path.join(ROOT, "include")
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libcmr.so")
+PROBE_DIR = os.path.join(PKG, "probe")
+PROBE_LIB = os.path.join(PKG, "libcmr_probe.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -30,23 +34,34 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def probe_sources():
+    return sorted(glob.glob(os.path.join(PROBE_DIR, "*.cu")))
+
+
+def _stale(lib, srcs) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "cmr.h"),
-                                                                  os.path.abspath(__file__)]
+    t = os.path.getmtime(lib)
+    deps = srcs + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "cmr.h"),
+                                                           os.path.abspath(__file__)]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
+def _nvcc(lib, srcs, verbose_ptxas):
+    tmp = lib + ".tmp.%d" % os.getpid()
     cmd = [NVCC] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + [
-        "-I", INCLUDE, "-o", tmp] + sources()
+        "-I", INCLUDE, "-o", tmp] + srcs
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    """Builds libcmr.so (and the probe library) when missing or older than
+    their sources; returns the path of libcmr.so."""
+    if force or _stale(LIB, sources()):
+        _nvcc(LIB, sources(), verbose_ptxas)
+    if force or _stale(PROBE_LIB, probe_sources()):
+        _nvcc(PROBE_LIB, probe_sources(), verbose_ptxas)
     return LIB
 
 

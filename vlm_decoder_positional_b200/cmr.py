@@ -31,6 +31,11 @@ SIGNATURES = {
     "cmr_positions_chunk": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
                                            ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
                                            _i32p, _i32p, _i32p, _i32p, ctypes.c_void_p]),
+    "cmr_positions_frames": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                            ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p,
+                                            ctypes.c_void_p, ctypes.c_size_t, _i32p,
+                                            ctypes.c_void_p]),
+    "cmr_positions_frames_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int64]),
     "cmr_positions_step": (ctypes.c_int, [_i32p, _i32p, _i32p, ctypes.c_int32, _i32p,
                                           ctypes.c_void_p]),
     "cmr_rotate_qk_shift": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p,
@@ -51,6 +56,12 @@ SIGNATURES = {
                                      ctypes.c_int32, ctypes.c_double,
                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32,
                                      _i32p, ctypes.c_void_p]),
+    "cmr_positions_rotate_qk": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                               ctypes.c_int32, _i32p, _i32p, _i32p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_double, ctypes.POINTER(ctypes.c_int32),
+                                               ctypes.c_int32, _i32p, ctypes.c_void_p]),
     "cmr_rotate_qk_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "cmr_rotate_qk_cache_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32,
@@ -61,6 +72,7 @@ SIGNATURES = {
                                              ctypes.c_void_p]),
     "cmr_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "cmr_last_error_message": (ctypes.c_char_p, []),
+    "cmr_last_rotate_kernel": (ctypes.c_char_p, []),
     "cmr_version": (ctypes.c_int32, []),
 }
 
@@ -210,6 +222,55 @@ def positions_chunk(ids: torch.Tensor, cu_seqlens: torch.Tensor,
                                          start.data_ptr() if b else None,
                                          amount.data_ptr() if b else None, st_ptr,
                                          _stream_ptr(dev, stream)), "cmr_positions_chunk")
+    return pos, start, amount
+
+
+def positions_frames_workspace_bytes(num_seqs: int, n_tokens: int) -> int:
+    """Workspace bytes cmr_positions_frames uses at full parallelism."""
+    return int(lib().cmr_positions_frames_workspace_bytes(int(num_seqs), int(n_tokens)))
+
+
+def positions_frames(ids: torch.Tensor, cu_seqlens: torch.Tensor, grid_side: int = 8,
+                     image_token_id: int = IMAGE_TOKEN_ID,
+                     out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     device_status: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None):
+    """cmr_positions_frames: planes of prompts in which every <image> marker
+    opens a frame on a grid_side x grid_side grid.  workspace: a CUDA tensor of
+    at least 16 bytes per sequence (allocated at full size when None).
+    Returns (pos [3, N], start [B], amount [B])."""
+    _want(ids, "ids", torch.int32)
+    dev = ids.device
+    _want(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    n, b = ids.numel(), cu_seqlens.numel() - 1
+    if b < 0:
+        raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+    if out is None:
+        pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+        start = torch.empty(b, dtype=torch.int32, device=dev)
+        amount = torch.empty(b, dtype=torch.int32, device=dev)
+    else:
+        pos, start, amount = out
+        for t, name in ((pos, "pos"), (start, "start"), (amount, "amount")):
+            _want(t, name, torch.int32, dev)
+        if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
+            raise ValueError("output shapes must be [3, N], [B], [B]")
+    if workspace is None:
+        workspace = torch.empty(max(positions_frames_workspace_bytes(b, n), 16),
+                                dtype=torch.uint8, device=dev)
+    if not workspace.is_cuda or workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor on the ids' device")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st_ptr = _status_ptr(device_status, dev)
+    with torch.cuda.device(dev):
+        _check(lib().cmr_positions_frames(ids.data_ptr() if n else None, cu_seqlens.data_ptr(),
+                                          b, n, int(image_token_id), int(grid_side),
+                                          pos.data_ptr() if n else None,
+                                          start.data_ptr() if b else None,
+                                          amount.data_ptr() if b else None,
+                                          workspace.data_ptr(), ws_bytes, st_ptr,
+                                          _stream_ptr(dev, stream)), "cmr_positions_frames")
     return pos, start, amount
 
 
@@ -387,6 +448,51 @@ def rotate_qk(q: Optional[torch.Tensor], k: Optional[torch.Tensor], pos: torch.T
                                    sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)),
                "cmr_rotate_qk")
     return q, k
+
+
+def positions_rotate_qk(ids: torch.Tensor, cu_seqlens: torch.Tensor, q: Optional[torch.Tensor],
+                        k: Optional[torch.Tensor], theta: float = 1e7,
+                        sections: Sequence[int] = (11, 11, 10), rot_dim: int = 64,
+                        image_token_id: int = IMAGE_TOKEN_ID,
+                        out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                        device_status: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None):
+    """cmr_positions_rotate_qk: positions, then the rotation of q and k in place
+    with those planes, the rotation overlapping the positions kernels.
+    Returns (pos [3, N], start [B], amount [B])."""
+    _want(ids, "ids", torch.int32)
+    dev = ids.device
+    _want(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    n, b = ids.numel(), cu_seqlens.numel() - 1
+    if b < 0:
+        raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+    L, hq, hk, D = _qk_shapes(q, k, dev, n)
+    if out is None:
+        pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+        start = torch.empty(b, dtype=torch.int32, device=dev)
+        amount = torch.empty(b, dtype=torch.int32, device=dev)
+    else:
+        pos, start, amount = out
+        for t, name in ((pos, "pos"), (start, "start"), (amount, "amount")):
+            _want(t, name, torch.int32, dev)
+        if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
+            raise ValueError("output shapes must be [3, N], [B], [B]")
+    st_ptr = _status_ptr(device_status, dev)
+    sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
+    with torch.cuda.device(dev):
+        _check(lib().cmr_positions_rotate_qk(
+            ids.data_ptr() if n else None, cu_seqlens.data_ptr(), b, n, int(image_token_id),
+            pos.data_ptr() if n else None, start.data_ptr() if b else None,
+            amount.data_ptr() if b else None,
+            q.data_ptr() if q is not None and q.numel() else None,
+            k.data_ptr() if k is not None and k.numel() else None, L, hq, hk, D, float(theta),
+            sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)), "cmr_positions_rotate_qk")
+    return pos, start, amount
+
+
+def last_rotate_kernel() -> str:
+    """Name of the rotate kernel this thread's last rotate call launched ('' before any)."""
+    return lib().cmr_last_rotate_kernel().decode()
 
 
 def rotate_qk_kernel(n_tokens: int, num_layers: int, hq: int, hk: int, head_dim: int = 256,

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <climits>
+#include <cstdint>
 #include <cstdio>
 
 #include "cmr.h"
@@ -12,6 +13,7 @@
 namespace {
 
 thread_local char g_message[320] = "no error";
+thread_local const char* g_last_kernel = nullptr;
 
 cmr_status fail(cmr_status s, const char* fmt, ...) {
   va_list ap;
@@ -111,28 +113,11 @@ cmr_status check_rotate(void* q, void* k, int64_t n_tokens, int32_t num_layers, 
   return CMR_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-const char* cmr_status_string(cmr_status s) {
-  switch (s) {
-    case CMR_OK: return "CMR_OK";
-    case CMR_EINVAL: return "CMR_EINVAL: invalid argument";
-    case CMR_ECUDA: return "CMR_ECUDA: CUDA runtime error";
-    case CMR_EUNSUPPORTED: return "CMR_EUNSUPPORTED: shape outside this build's limits";
-  }
-  return "unknown cmr_status";
-}
-
-const char* cmr_last_error_message(void) { return g_message; }
-
-int32_t cmr_version(void) { return 20000; }  // 2.0.0
-
-cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
-                         int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
-                         int32_t* out_start, int32_t* out_amount, int32_t* device_status,
-                         cmr_stream_t stream) {
+// Checks of cmr_positions' arguments (num_seqs == 0 with no tokens is valid
+// and leaves nothing to do).
+cmr_status check_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                           int64_t n_tokens, const int32_t* out_pos, const int32_t* out_start,
+                           const int32_t* out_amount, const int32_t* device_status) {
   if (num_seqs < 0 || n_tokens < 0) return fail(CMR_EINVAL, "negative num_seqs or n_tokens");
   if (n_tokens > INT32_MAX) return fail(CMR_EINVAL, "n_tokens exceeds int32 indexing");
   if (num_seqs == 0) {
@@ -151,6 +136,40 @@ cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t 
     if ((s = check_device_ptr(out_pos, "out_pos")) != CMR_OK) return s;
   }
   if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  return CMR_OK;
+}
+
+}  // namespace
+
+namespace cmr {
+void note_kernel(const char* name) { g_last_kernel = name; }
+}  // namespace cmr
+
+extern "C" {
+
+const char* cmr_status_string(cmr_status s) {
+  switch (s) {
+    case CMR_OK: return "CMR_OK";
+    case CMR_EINVAL: return "CMR_EINVAL: invalid argument";
+    case CMR_ECUDA: return "CMR_ECUDA: CUDA runtime error";
+    case CMR_EUNSUPPORTED: return "CMR_EUNSUPPORTED: shape outside this build's limits";
+  }
+  return "unknown cmr_status";
+}
+
+const char* cmr_last_error_message(void) { return g_message; }
+
+const char* cmr_last_rotate_kernel(void) { return g_last_kernel ? g_last_kernel : ""; }
+
+int32_t cmr_version(void) { return 20100; }  // 2.1.0
+
+cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                         int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
+                         int32_t* out_start, int32_t* out_amount, int32_t* device_status,
+                         cmr_stream_t stream) {
+  cmr_status s = check_positions(ids, cu_seqlens, num_seqs, n_tokens, out_pos, out_start,
+                                 out_amount, device_status);
+  if (s != CMR_OK || num_seqs == 0) return s;
   cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
                                         CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
                                         out_start, out_amount, device_status,
@@ -202,6 +221,36 @@ cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seqlens, in
   return CMR_OK;
 }
 
+size_t cmr_positions_frames_workspace_bytes(int32_t num_seqs, int64_t n_tokens) {
+  if (num_seqs <= 0 || n_tokens < 0) return 0;
+  return static_cast<size_t>(cmr::frames_slices(num_seqs, n_tokens, SIZE_MAX)) *
+         cmr::frames_summary_bytes() * static_cast<size_t>(num_seqs);
+}
+
+cmr_status cmr_positions_frames(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
+                                int64_t n_tokens, int32_t image_token_id, int32_t grid_side,
+                                int32_t* out_pos, int32_t* out_start, int32_t* out_amount,
+                                void* workspace, size_t workspace_bytes,
+                                int32_t* device_status, cmr_stream_t stream) {
+  if (grid_side < 1 || grid_side > 128) return fail(CMR_EINVAL, "grid_side must be in 1 .. 128");
+  cmr_status s = check_positions(ids, cu_seqlens, num_seqs, n_tokens, out_pos, out_start,
+                                 out_amount, device_status);
+  if (s != CMR_OK || num_seqs == 0) return s;
+  const size_t one = cmr::frames_summary_bytes() * static_cast<size_t>(num_seqs);
+  if (!workspace || workspace_bytes < one)
+    return fail(CMR_EINVAL, "workspace must hold at least %zu bytes (16 per sequence)", one);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return fail(CMR_EINVAL, "workspace must be 16-byte aligned");
+  if ((s = check_device_ptr(workspace, "workspace")) != CMR_OK) return s;
+  cudaError_t e = cmr::launch_positions_frames(ids, cu_seqlens, num_seqs, n_tokens,
+                                               image_token_id, grid_side, out_pos, out_start,
+                                               out_amount, workspace, workspace_bytes,
+                                               device_status,
+                                               reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions_frames launch");
+  return CMR_OK;
+}
+
 cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* start,
                               const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
                               cmr_stream_t stream) {
@@ -235,6 +284,38 @@ cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n_tokens,
   a.pos = pos;
   a.status = device_status;
   cudaError_t e = cmr::launch_rotate_qk(a, table, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_positions_rotate_qk(const int32_t* ids, const int32_t* cu_seqlens,
+                                   int32_t num_seqs, int64_t n_tokens, int32_t image_token_id,
+                                   int32_t* out_pos, int32_t* out_start, int32_t* out_amount,
+                                   void* q, void* k, int32_t num_layers, int32_t hq, int32_t hk,
+                                   int32_t head_dim, double theta, const int32_t sections[3],
+                                   int32_t rot_dim, int32_t* device_status,
+                                   cmr_stream_t stream) {
+  // Every check of both steps runs before anything is enqueued.
+  cmr::RotateArgs a;
+  cmr::FreqTable table;
+  cmr_status s = check_positions(ids, cu_seqlens, num_seqs, n_tokens, out_pos, out_start,
+                                 out_amount, device_status);
+  if (s != CMR_OK) return s;
+  s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections, rot_dim, &a,
+                   &table);
+  if (s != CMR_OK) return s;
+  if (num_seqs == 0) return CMR_OK;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
+                                        CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
+                                        out_start, out_amount, device_status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "positions launch");
+  if (a.n_tokens == 0) return CMR_OK;
+  a.pos = out_pos;
+  a.status = device_status;
+  // The rotation follows the positions kernels directly, so it may start
+  // while they finish: its Q/K loads do not depend on them.
+  e = cmr::launch_rotate_qk(a, table, st, /*programmatic=*/true);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
   return CMR_OK;
 }

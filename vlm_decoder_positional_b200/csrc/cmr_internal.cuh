@@ -82,11 +82,27 @@ cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int3
                              const int32_t* in_amount, int32_t* out_pos, int32_t* out_start,
                              int32_t* out_amount, int32_t* device_status, cudaStream_t stream);
 
+// Multi-frame canvas (frames.cu): slices per prompt for a workspace of
+// `workspace_bytes` (0 when not even one summary per prompt fits), the bytes of
+// one slice summary, and the launch of the summary and planes kernels.
+int64_t frames_slices(int32_t num_seqs, int64_t n_tokens, size_t workspace_bytes);
+size_t frames_summary_bytes();
+cudaError_t launch_positions_frames(const int32_t* ids, const int32_t* cu_seqlens,
+                                    int32_t num_seqs, int64_t n_tokens, int32_t image_token_id,
+                                    int32_t grid_side, int32_t* out_pos, int32_t* out_start,
+                                    int32_t* out_amount, void* workspace,
+                                    size_t workspace_bytes, int32_t* device_status,
+                                    cudaStream_t stream);
+
 cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start,
                                   const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
                                   cudaStream_t stream);
 
-cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream);
+// programmatic: launch with programmatic stream serialization, which only a
+// launch that directly follows this library's positions kernels may ask for:
+// the staged kernel's Q/K loads start before the wait for pos.
+cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream,
+                             bool programmatic = false);
 
 // TMA tensor map of a bf16 tensor: dims[0] is contiguous, strides_bytes[i] is
 // the byte stride of dims[i + 1] (any order), box[i] the box extent per dim.
@@ -94,6 +110,10 @@ cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cud
 bool encode_bf16_tensor_map(CUtensorMap* map, void* base, int rank, const uint64_t* dims,
                             const uint64_t* strides_bytes, const uint32_t* box,
                             bool swizzle_128b);
+// Records, per calling thread, the name of the rotate kernel a launch enqueued
+// (read back through cmr_last_rotate_kernel).
+void note_kernel(const char* name);
+
 // L2 size of the current device in bytes (cached; 0 if it cannot be read).
 int64_t device_l2_bytes();
 
@@ -105,6 +125,6 @@ bool staged_rotate_fits(const RotateArgs& args);
 bool rotate_qk_uses_staged(const RotateArgs& args);
 int64_t staged_rotate_tiles(int64_t n_tokens);
 cudaError_t launch_rotate_qk_staged(const RotateArgs& args, const FreqTable& table,
-                                    cudaStream_t stream, bool* launched);
+                                    cudaStream_t stream, bool programmatic, bool* launched);
 
 }  // namespace cmr

@@ -34,6 +34,7 @@
 // each computing the same 8 cos/sin.
 #include <mutex>
 
+#include "pdl.cuh"
 #include "rotate_common.cuh"
 
 namespace cmr {
@@ -100,6 +101,9 @@ __global__ void __launch_bounds__(kThreads, BatchShape<kBatch>::kMinBlocksPerSm)
   // Planes of the current item's token, loaded one item ahead so that their
   // latency overlaps the previous item's head rows.
   int32_t p0 = 0, p1 = 0, p2 = 0;
+  // Launched programmatically behind the positions kernels, pos is only
+  // ready after this wait; otherwise it returns at once.
+  if constexpr (!kFromShift) pdl::wait();
   if (v < n_items) token_planes<kFromShift>(args, G == 1 ? v : v % N, p0, p1, p2);
   for (; v < n_items; v += v_step) {
     const int64_t g = (G == 1) ? 0 : v / N;
@@ -228,10 +232,11 @@ bool rotate_qk_uses_staged(const RotateArgs& a) {
   return staged_rotate_tiles(a.n_tokens) >= kMinStagedTiles && staged_rotate_fits(a);
 }
 
-cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream) {
+cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaStream_t stream,
+                             bool programmatic) {
   if (rotate_qk_uses_staged(in)) {
     bool launched = false;
-    const cudaError_t e = launch_rotate_qk_staged(in, table, stream, &launched);
+    const cudaError_t e = launch_rotate_qk_staged(in, table, stream, programmatic, &launched);
     if (e != cudaSuccess || launched) return e;
   }
   RotateArgs a = in;
@@ -256,9 +261,10 @@ cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaS
   const int64_t items = a.n_tokens * a.job_groups;
   const int64_t needed = (items + items_per_cta - 1) / items_per_cta;
   const int64_t ctas = (plan.one_shot || needed <= max_ctas) ? needed : max_ctas;
-  variant(from_shift, plan.batch_index)<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(
-      a, table);
-  return cudaGetLastError();
+  e = pdl::launch(variant(from_shift, plan.batch_index), dim3(static_cast<unsigned>(ctas)),
+                  dim3(kThreads), 0, stream, programmatic, a, table);
+  if (e == cudaSuccess) note_kernel("rotate_qk_kernel");
+  return e;
 }
 
 }  // namespace cmr

@@ -237,7 +237,9 @@ cudaError_t launch_rotate_qk_cache(const CacheArgs& in, const FreqTable& table,
   // in one moving window.
   const int64_t ctas = needed;
   rotate_qk_cache_kernel<<<static_cast<unsigned>(ctas), kThreads, 0, stream>>>(ca, table);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) note_kernel("rotate_qk_cache_kernel");
+  return e;
 }
 
 }  // namespace cmr

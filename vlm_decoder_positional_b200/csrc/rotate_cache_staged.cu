@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(kThreads)
   int st = 0, prev = S - 1;
   uint32_t phase = 0;
   for (int l = 0; l < L; ++l) {
-    const bool landed = tma::mbar_wait(full0 + 8 * st, phase);
+    const bool landed = tma::mbar_wait(full0 + 8 * st, phase, tma::kConsumerWaitLimitNs);
     if (tma::named_any(1, kConsumers, !landed)) {
       if (threadIdx.x == 0) report(status, CMR_DEVICE_WAIT_TIMEOUT);
       break;
@@ -295,9 +295,13 @@ cudaError_t launch_rotate_qk_cache_staged(const CacheArgs& ca, const FreqTable& 
     if (!g_smem_set[dev & 63]) {
       // The opt-in is an attribute call, which a stream capture may forbid:
       // a first launch inside a capture takes the register kernel instead.
+      // The query itself fails on the legacy stream while another stream
+      // captures in global mode; that launch takes the register kernel too.
       cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-      e = cudaStreamIsCapturing(stream, &cap);
-      if (e != cudaSuccess) return e;
+      if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+      }
       if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
       e = cudaFuncSetAttribute(rotate_qk_cache_staged_kernel,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -315,7 +319,10 @@ cudaError_t launch_rotate_qk_cache_staged(const CacheArgs& ca, const FreqTable& 
   rotate_qk_cache_staged_kernel<<<static_cast<unsigned>(ctas), kThreads, smem, stream>>>(
       q_map, k_map, v_map, kc_map, vc_map, sa, table);
   e = cudaGetLastError();
-  if (e == cudaSuccess) *launched = true;
+  if (e == cudaSuccess) {
+    *launched = true;
+    note_kernel("rotate_qk_cache_staged_kernel");
+  }
   return e;
 }
 

@@ -34,6 +34,7 @@
 // the loads it issued, and returns.
 #include <mutex>
 
+#include "pdl.cuh"
 #include "rotate_common.cuh"
 #include "tma.cuh"
 
@@ -143,6 +144,10 @@ __global__ void __launch_bounds__(kThreads)
   const int tl = (threadIdx.x >> 5) * 8 + ((lane >> 3) | (((lane >> 2) & 1) << 2));
   const int64_t t = static_cast<int64_t>(t0) + tl;
   int32_t p0 = 0, p1 = 0, p2 = 0;  // rows past the last token are zeros and are not stored
+  // Launched programmatically behind the positions kernels, the producer's
+  // loads of Q and K (which those kernels never touch) are already under way;
+  // pos is ready after this wait.  Otherwise it returns at once.
+  if constexpr (!kFromShift) pdl::wait();
   if (t < args.r.n_tokens) token_planes<kFromShift>(args.r, t, p0, p1, p2);
   float c[8], s[8];
 #pragma unroll
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(kThreads)
   int st = 0, prev = S - 1;  // this layer's stage and the previous layer's
   uint32_t phase = 0;        // (l / S) & 1
   for (int l = 0; l < L; ++l) {
-    const bool landed = tma::mbar_wait(full0 + 8 * st, phase);
+    const bool landed = tma::mbar_wait(full0 + 8 * st, phase, tma::kConsumerWaitLimitNs);
     if (tma::named_any(1, kConsumers, !landed)) {
       if (threadIdx.x == 0) report_timeout(args.r.status);
       break;
@@ -239,7 +244,7 @@ int64_t staged_rotate_tiles(int64_t n_tokens) { return (n_tokens + kTileTokens -
 // Launch the staged kernel; *launched is false (and nothing was enqueued)
 // when the tensor maps cannot describe these buffers.
 cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
-                                    cudaStream_t stream, bool* launched) {
+                                    cudaStream_t stream, bool programmatic, bool* launched) {
   *launched = false;
   CUtensorMap q_map{}, k_map{};
   if (a.hq > 0 && !encode_map(&q_map, a.q, a.n_tokens, a.hq, a.num_layers, a.head_dim))
@@ -267,9 +272,13 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
     if (!done && smem > 48 * 1024) {
       // a capture may forbid the attribute call: that first launch takes the
       // register kernel instead
+      // The query itself fails on the legacy stream while another stream
+      // captures in global mode; that launch takes the register kernel too.
       cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-      e = cudaStreamIsCapturing(stream, &cap);
-      if (e != cudaSuccess) return e;
+      if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+      }
       if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(1024 + kStages * (kMaxStageBytes + 16)));
@@ -289,9 +298,12 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
                         static_cast<int64_t>(kRowBytes);
   sa.evict_first = moved <= kEvictFirstL2Multiple * l2_bytes ? 1 : 0;
   const int64_t tiles = staged_rotate_tiles(a.n_tokens);
-  fn<<<static_cast<unsigned>(tiles), kThreads, smem, stream>>>(q_map, k_map, sa, table);
-  e = cudaGetLastError();
-  if (e == cudaSuccess) *launched = true;
+  e = pdl::launch(fn, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), smem, stream,
+                  programmatic, q_map, k_map, sa, table);
+  if (e == cudaSuccess) {
+    *launched = true;
+    note_kernel("rotate_qk_staged_kernel");
+  }
   return e;
 }
 

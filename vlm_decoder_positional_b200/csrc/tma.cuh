@@ -15,6 +15,17 @@ namespace tma {
 // here last microseconds.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
+// Limit of the consumers' waits for a stage's data.  Builds of the library
+// use kWaitLimitNs; the time-out test compiles a separate copy with
+// -DCMR_CONSUMER_WAIT_LIMIT_NS=0, so that these waits give up on ordinary
+// copies and the time-out path runs, while the producer's drain keeps the
+// full limit and still sees every load it issued land.
+#ifdef CMR_CONSUMER_WAIT_LIMIT_NS
+constexpr uint64_t kConsumerWaitLimitNs = CMR_CONSUMER_WAIT_LIMIT_NS;
+#else
+constexpr uint64_t kConsumerWaitLimitNs = kWaitLimitNs;
+#endif
+
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -58,13 +69,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait for the phase of parity `parity` to complete; false after
-// kWaitLimitNs without it.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of parity `parity` to complete; false after `limit_ns`
+// without it.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (!mbar_try_wait(bar, parity))
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   return true;
 }
 

@@ -181,11 +181,13 @@ CONFIG_NAMES = {
     3: "c3_64x4096_outliers",
     4: "c4_decode_1024",
     5: "c5_6layers_32x8192",
+    6: "c6_multiframe_256x65536",  # the multi-frame positions' workload (not a rotate config)
 }
 
 
 def make_config(index: int, device="cpu", with_qk=True, seed=None) -> Workload:
-    """The five synthetic workloads (1-based index, seed = 20261013 + index)."""
+    """The five synthetic workloads (1-based index, seed = 20261013 + index), and
+    6: the multi-frame positions' workload (make_frames_workload)."""
     seed = BASE_SEED + index if seed is None else seed
     rng = np.random.default_rng(seed)
     name = CONFIG_NAMES[index]
@@ -224,4 +226,36 @@ def make_config(index: int, device="cpu", with_qk=True, seed=None) -> Workload:
         origins = rng.integers(0, 6001, size=32)
         return make_batch([8192] * 32, origins, num_layers=6, seed=seed, device=device,
                           with_qk=with_qk, name=name)
-    raise ValueError("config index must be 1..5")
+    if index == 6:
+        return make_frames_workload(seed=seed, device=device)  # positions only: no Q/K
+    raise ValueError("config index must be 1..6")
+
+
+def make_frames_workload(num_prompts=256, length=65536, frames=32, grid_side=8, seed=None,
+                         device="cpu", with_qk=False, min_text=16) -> Workload:
+    """Prompts that each hold several frames on a grid_side x grid_side grid (a
+    thumbnail and its slices, or several images), with at least ``min_text``
+    text tokens between frames: the workload of the multi-frame positions.
+    The default, 256 prompts x 65,536 tokens with 32 frames each (16.8 M
+    tokens, 268 MB of ids and planes), is larger than the L2.  Q/K are not
+    drawn unless asked for (one layer)."""
+    seed = BASE_SEED + 6 if seed is None else seed
+    rng = np.random.default_rng(seed)
+    F = grid_side * grid_side + 3
+    prompts, first = [], []
+    for _ in range(num_prompts):
+        origins = spaced_origins(rng, frames, 0, length - F, F + min_text)
+        prompts.append(prompt_ids_frames(rng, length, origins, grid_side))
+        first.append(origins[0])
+    ids, cu = pack(prompts)
+    n = ids.shape[0]
+    q = k = None
+    if with_qk:
+        q = random_qk((1, n, HQ, HEAD_DIM), seed + 1, device)
+        k = random_qk((1, n, HK, HEAD_DIM), seed + 2, device)
+    name = (f"c6_multiframe_{num_prompts}x{length}_{frames}frames_s{grid_side}"
+            if (num_prompts, length, frames, grid_side) != (256, 65536, 32, 8)
+            else CONFIG_NAMES[6])
+    return Workload(name=name, ids=ids, cu_seqlens=cu,
+                    frame_origin=np.array(first, dtype=np.int32), q=q, k=k, seed=seed,
+                    meta={"grid_side": grid_side, "frames_per_prompt": frames})

@@ -3,7 +3,8 @@
 For callers whose ids and Q/K live in (pinned) host memory.  The batch is cut
 into chunks of whole prompts (a prompt is never split, so each chunk's planes
 need nothing from another chunk).  Each chunk goes host -> device on one stream,
-through cmr_positions + cmr_rotate_qk on a second, and back on a third, over a
+through cmr_positions_rotate_qk (the positions kernels, then the rotation
+overlapping them) on a second, and back on a third, over a
 ring of `depth` device buffers, so the host-to-device copy of one chunk, the
 kernels of the next and the device-to-host copy of a third run at the same
 time (PCIe moves both directions at once).  Only the rotated dims of each head
@@ -105,9 +106,9 @@ class HostPipeline:
                 self.copied_in[r].record(self.s_in)
             with torch.cuda.stream(self.s_run):
                 self.s_run.wait_event(self.copied_in[r])
-                cmr.positions(self.ids[r][:n], self.cu[r][:b + 1], image_token_id,
-                              out=(pos_d, self.start[r][:b], self.amount[r][:b]))
-                cmr.rotate_qk(q_d, k_d, pos_d, theta, sections, rot_dim)
+                cmr.positions_rotate_qk(self.ids[r][:n], self.cu[r][:b + 1], q_d, k_d, theta,
+                                        sections, rot_dim, image_token_id,
+                                        out=(pos_d, self.start[r][:b], self.amount[r][:b]))
                 self.computed[r].record(self.s_run)
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(self.computed[r])
