@@ -94,11 +94,10 @@ typedef enum cmr_status {
  *                and write no planes for the prompts whose bounds are invalid
  *                (their out_start / out_amount entries are then unspecified).
  *                The library never clears it.
- * The work is a memset of out_start and two kernels: a scan of each slice of
- * each prompt for its first marker, which lowers out_start[b] with an atomic
- * min (every id is read once), then the planes and the state.  out_start is
- * therefore written during the call; it must not be read or written by other
- * work in flight.
+ * Two kernels: one CTA per prompt scans its ids up to the first marker (no
+ * id is read twice) and writes the state; then CTAs over slices of about
+ * 2,048 tokens write the planes, reading the state back from out_start /
+ * out_amount.
  * Errors: CMR_EINVAL for null required pointers, negative sizes, num_seqs = 0
  * with n_tokens > 0, or n_tokens > INT32_MAX. */
 CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,
@@ -246,14 +245,18 @@ CMR_API cmr_status cmr_rotate_qk(void* q, void* k, const int32_t* pos, int64_t n
                          const int32_t sections[3], int32_t rot_dim,
                          int32_t* device_status, cmr_stream_t stream);
 
-/* The whole path in one call: cmr_positions, then cmr_rotate_qk with the
- * planes just written (same arguments, same results, bit for bit).  The
- * rotation is launched with programmatic stream serialization behind the
- * positions kernels: its CTAs start while the planes are being written, the
- * TMA loads of Q and K (which the positions kernels never touch) go out at
- * once, and only the rotation itself waits for the planes.  Launching the
- * two separately cannot overlap them, because a caller's kernel before a
- * plain cmr_rotate_qk may still be writing Q/K when it signals.
+/* The whole path in one call: the results of cmr_positions and then
+ * cmr_rotate_qk with those planes (same arguments, same results, bit for
+ * bit).  Two kernels: the origin scan writes each prompt's (start, amount);
+ * the rotation is launched with programmatic stream serialization behind it,
+ * so its CTAs start while the scan runs and the TMA loads of Q and K (which
+ * the scan never touches) go out at once; it then derives each token's planes
+ * from its prompt's state, writes them to out_pos and rotates with them.
+ * Launching the two calls separately cannot overlap them, because a caller's
+ * kernel before a plain cmr_rotate_qk may still be writing Q/K when it
+ * signals.  With no layers to rotate, the planes kernel of cmr_positions
+ * writes out_pos instead.  With malformed cu_seqlens the planes and rows of
+ * the prompts involved are unspecified (CMR_DEVICE_BAD_CU_SEQLENS is set).
  *
  *   ids, cu_seqlens, num_seqs, n_tokens, image_token_id, out_pos, out_start,
  *   out_amount     as in cmr_positions (out_pos is also the rotation's pos)

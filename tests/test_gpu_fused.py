@@ -92,3 +92,28 @@ def test_one_call_replayed_from_a_cuda_graph(cuda_device, shape, kernel):
         BarStats("graph q").add(bits(q), oracle_rotate_threads(q_in, want_pos)).check()
         BarStats("graph k").add(bits(k), oracle_rotate_threads(k_in, want_pos)).check()
     assert int(status.item()) == 0
+
+
+def test_one_call_with_empty_prompts_and_without_layers(cuda_device):
+    # empty prompts get their state from the origin scan alone; with no
+    # layers to rotate the planes kernel writes pos
+    dev = cuda_device
+    rng = np.random.default_rng(9)
+    prompts = [np.zeros(0, np.int32), inputs.prompt_ids(rng, 5000, 17), np.zeros(0, np.int32),
+               inputs.prompt_ids(rng, 4000, -1), inputs.prompt_ids(rng, 3000, 2990)]
+    ids_np, cu_np = inputs.pack(prompts)
+    ids, cu = t32(ids_np, dev), t32(cu_np, dev)
+    n = ids_np.shape[0]
+    want = oracle.positions(ids_np, cu_np)
+    for layers in (0, 1, 3):
+        q = inputs.random_qk((layers, n, 8, 256), 40 + layers, dev) if layers else \
+            torch.empty((0, n, 8, 256), dtype=torch.bfloat16, device=dev)
+        k = inputs.random_qk((layers, n, 2, 256), 50 + layers, dev) if layers else \
+            torch.empty((0, n, 2, 256), dtype=torch.bfloat16, device=dev)
+        q_in = bits(q)
+        got = cmr.positions_rotate_qk(ids, cu, q, k)
+        torch.cuda.synchronize()
+        for g, w in zip(got, want):
+            np.testing.assert_array_equal(g.cpu().numpy(), w)
+        if layers:
+            BarStats(f"q L={layers}").add(bits(q), oracle_rotate_threads(q_in, want[0])).check()

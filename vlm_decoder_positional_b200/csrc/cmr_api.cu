@@ -306,15 +306,28 @@ cmr_status cmr_positions_rotate_qk(const int32_t* ids, const int32_t* cu_seqlens
   if (s != CMR_OK) return s;
   if (num_seqs == 0) return CMR_OK;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
-                                        CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
-                                        out_start, out_amount, device_status, st);
+  if (a.n_tokens == 0) {  // no rotation (no layers): the planes kernel writes pos
+    cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
+                                          CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
+                                          out_start, out_amount, device_status, st);
+    return e == cudaSuccess ? CMR_OK : cuda_fail(e, "positions launch");
+  }
+  // The origin scan writes each prompt's (start, amount); the rotation,
+  // launched to start while the scan runs (its Q/K loads do not depend on it),
+  // derives each token's planes from that state, writes them to out_pos and
+  // rotates -- the planes kernel is not needed.
+  cudaError_t e = cmr::launch_positions_origin(ids, cu_seqlens, num_seqs, n_tokens,
+                                               image_token_id, CMR_RULE_CANVAS, nullptr, nullptr,
+                                               nullptr, out_start, out_amount, device_status, st);
   if (e != cudaSuccess) return cuda_fail(e, "positions launch");
-  if (a.n_tokens == 0) return CMR_OK;
-  a.pos = out_pos;
+  a.pos = nullptr;
+  a.cu = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.pos_offset = nullptr;
+  a.start = out_start;
+  a.amount = out_amount;
+  a.pos_out = out_pos;
   a.status = device_status;
-  // The rotation follows the positions kernels directly, so it may start
-  // while they finish: its Q/K loads do not depend on them.
   e = cmr::launch_rotate_qk(a, table, st, /*programmatic=*/true);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
   return CMR_OK;

@@ -43,6 +43,9 @@ struct RotateArgs {
   int32_t num_layers;
   int32_t hq, hk, head_dim, rot_dim;
   int32_t* status;         // optional device status word (staged kernel time-outs)
+  // with the shift state: also write each token's planes to pos_out [3, N]
+  // (the one-call path, where the rotation replaces the planes kernel)
+  int32_t* pos_out;
   int32_t units_per_head;  // rot_dim / 16: threads per token, 8 frequencies each
   int32_t job_groups;       // work items per token (set at launch)
   int32_t jobs_per_group;   // (layer, head) rows per work item
@@ -75,6 +78,14 @@ cudaError_t launch_rotate_qk_cache(const CacheArgs& args, const FreqTable& table
 bool rotate_qk_cache_uses_staged(const RotateArgs& args);
 cudaError_t launch_rotate_qk_cache_staged(const CacheArgs& args, const FreqTable& table,
                                           cudaStream_t stream, bool* launched);
+
+// The origin kernel alone: each chunk's outgoing (start, amount), no planes.
+cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlens,
+                                   int32_t num_seqs, int64_t n_tokens, int32_t image_token_id,
+                                   int32_t rule, const int32_t* pos_offset,
+                                   const int32_t* in_start, const int32_t* in_amount,
+                                   int32_t* out_start, int32_t* out_amount,
+                                   int32_t* device_status, cudaStream_t stream);
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                              int64_t n_tokens, int32_t image_token_id, int32_t rule,

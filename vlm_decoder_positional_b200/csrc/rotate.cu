@@ -101,13 +101,15 @@ __global__ void __launch_bounds__(kThreads, BatchShape<kBatch>::kMinBlocksPerSm)
   // Planes of the current item's token, loaded one item ahead so that their
   // latency overlaps the previous item's head rows.
   int32_t p0 = 0, p1 = 0, p2 = 0;
-  // Launched programmatically behind the positions kernels, pos is only
-  // ready after this wait; otherwise it returns at once.
-  if constexpr (!kFromShift) pdl::wait();
+  // Launched programmatically behind the positions kernels, pos (or the
+  // shift state) is only ready after this wait; otherwise it returns at once.
+  pdl::wait();
   if (v < n_items) token_planes<kFromShift>(args, G == 1 ? v : v % N, p0, p1, p2);
   for (; v < n_items; v += v_step) {
     const int64_t g = (G == 1) ? 0 : v / N;
     const int64_t t = v - g * N;
+    if (kFromShift && args.pos_out != nullptr && u == 0 && g == 0)
+      store_planes(args, t, p0, p1, p2);
     const int j_lo = static_cast<int>(g) * jpg;
     const int rows = min(J, j_lo + jpg) - j_lo;
     // Base of this thread's unit in head 0 of layer 0; K rows are indexed by

@@ -75,6 +75,14 @@ __device__ __forceinline__ void token_seq(const RotateArgs& a, int64_t t, int32_
   p = (a.pos_offset ? __ldg(a.pos_offset + b) : 0) + local;
 }
 
+// The one-call path's rotation writes the planes of token t that it derived.
+__device__ __forceinline__ void store_planes(const RotateArgs& a, int64_t t, int32_t p0,
+                                             int32_t p1, int32_t p2) {
+  a.pos_out[t] = p0;
+  a.pos_out[a.n_tokens + t] = p1;
+  a.pos_out[2 * a.n_tokens + t] = p2;
+}
+
 template <bool kFromShift>
 __device__ __forceinline__ void token_planes(const RotateArgs& a, int64_t t, int32_t& p0,
                                              int32_t& p1, int32_t& p2) {
@@ -86,7 +94,9 @@ __device__ __forceinline__ void token_planes(const RotateArgs& a, int64_t t, int
     int32_t b;
     int64_t p;
     token_seq(a, t, b, p);
-    const Planes r = canvas_row(p, __ldg(a.start + b), __ldg(a.amount + b));
+    // start / amount may come from the kernel just before (the one-call
+    // path's origin scan): read through L2, not the read-only path
+    const Planes r = canvas_row(p, __ldcg(a.start + b), __ldcg(a.amount + b));
     p0 = r.t;
     p1 = r.h;
     p2 = r.w;

@@ -146,9 +146,13 @@ __global__ void __launch_bounds__(kThreads)
   int32_t p0 = 0, p1 = 0, p2 = 0;  // rows past the last token are zeros and are not stored
   // Launched programmatically behind the positions kernels, the producer's
   // loads of Q and K (which those kernels never touch) are already under way;
-  // pos is ready after this wait.  Otherwise it returns at once.
-  if constexpr (!kFromShift) pdl::wait();
-  if (t < args.r.n_tokens) token_planes<kFromShift>(args.r, t, p0, p1, p2);
+  // pos (or the shift state) is ready after this wait.  Otherwise it returns
+  // at once.
+  pdl::wait();
+  if (t < args.r.n_tokens) {
+    token_planes<kFromShift>(args.r, t, p0, p1, p2);
+    if (kFromShift && args.r.pos_out != nullptr && u == 0) store_planes(args.r, t, p0, p1, p2);
+  }
   float c[8], s[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -258,34 +262,6 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
   sa.stage_bytes = sa.q_box_bytes + sa.k_box_bytes;
   sa.stages = a.num_layers < kStages ? a.num_layers : kStages;
   const bool from_shift = a.pos == nullptr;
-  const StagedFn fn = from_shift ? rotate_qk_staged_kernel<true> : rotate_qk_staged_kernel<false>;
-  const size_t smem = 1024 + static_cast<size_t>(sa.stages) * (sa.stage_bytes + 16);
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  {
-    std::lock_guard<std::mutex> lock(g_dev.mu);
-    // Only shapes whose ring exceeds the default 48 KB of dynamic shared
-    // memory need the opt-in (10 KB stages of 8 + 2 heads never do), so the
-    // common launch makes no attribute call, inside a graph capture or not.
-    bool& done = g_dev.smem_set[dev & 63][from_shift ? 1 : 0];
-    if (!done && smem > 48 * 1024) {
-      // a capture may forbid the attribute call: that first launch takes the
-      // register kernel instead
-      // The query itself fails on the legacy stream while another stream
-      // captures in global mode; that launch takes the register kernel too.
-      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-      if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
-        cudaGetLastError();
-        return cudaSuccess;
-      }
-      if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(1024 + kStages * (kMaxStageBytes + 16)));
-      if (e != cudaSuccess) return e;
-      done = true;
-    }
-  }
   const int64_t l2_bytes = device_l2_bytes();
   // L2 policy.  A launch that moves a few L2 sizes or less ends with most of
   // its rows still dirty in L2, and whatever reads them next competes with
@@ -298,6 +274,35 @@ cudaError_t launch_rotate_qk_staged(const RotateArgs& a, const FreqTable& table,
                         static_cast<int64_t>(kRowBytes);
   sa.evict_first = moved <= kEvictFirstL2Multiple * l2_bytes ? 1 : 0;
   const int64_t tiles = staged_rotate_tiles(a.n_tokens);
+  cudaError_t e;
+  const StagedFn fn = from_shift ? rotate_qk_staged_kernel<true> : rotate_qk_staged_kernel<false>;
+  const size_t smem = 1024 + static_cast<size_t>(sa.stages) * (sa.stage_bytes + 16);
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lock(g_dev.mu);
+    // Only shapes whose ring exceeds the default 48 KB of dynamic shared
+    // memory need the opt-in (10 KB stages of 8 + 2 heads never do), so the
+    // common launch makes no attribute call, inside a graph capture or not.
+    bool& done = g_dev.smem_set[dev & 63][from_shift ? 1 : 0];
+    if (!done && smem > 48 * 1024) {
+      // A capture may forbid the attribute call: that first launch takes the
+      // register kernel instead.  The query itself fails on the legacy stream
+      // while another stream captures in global mode; that launch takes the
+      // register kernel too.
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+        cudaGetLastError();
+        return cudaSuccess;
+      }
+      if (cap != cudaStreamCaptureStatusNone) return cudaSuccess;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(1024 + kStages * (kMaxStageBytes + 16)));
+      if (e != cudaSuccess) return e;
+      done = true;
+    }
+  }
   e = pdl::launch(fn, dim3(static_cast<unsigned>(tiles)), dim3(kThreads), smem, stream,
                   programmatic, q_map, k_map, sa, table);
   if (e == cudaSuccess) {
