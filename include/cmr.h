@@ -192,6 +192,34 @@ CMR_API cmr_status cmr_positions_frames(const int32_t* ids, const int32_t* cu_se
  * sequences).  No CUDA call is made. */
 CMR_API size_t cmr_positions_frames_workspace_bytes(int32_t num_seqs, int64_t n_tokens);
 
+/* cmr_positions_frames for callers that cannot allocate device memory and so
+ * cannot hand over a workspace: code running while a CUDA graph is being
+ * captured (cudaMalloc is refused there), serving loops that forbid
+ * allocation on the hot path (cudaMalloc may synchronise the device and its
+ * latency is unbounded), and plug-ins whose host application owns all device
+ * memory through its own allocator.  Same arguments, results and errors as
+ * cmr_positions_frames, without the workspace: the slice summaries live in a
+ * scratch array built into the library, 256 KB (16,384 summaries of 16
+ * bytes) that every device loading the library holds until the process
+ * exits.  It serves up to 16,384 sequences per call (more: CMR_EINVAL, and
+ * cmr_positions_frames with a workspace is the way); the more sequences, the
+ * fewer and longer the slices each prompt is split into.
+ *   - The first call on each device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing any stream into a CUDA graph.
+ *   - Every call on a device shares the one scratch: calls that overlap on
+ *     the device (other streams, other host threads) race and must be
+ *     serialised by the caller.  A call writes every summary it reads, so
+ *     nothing is left to clear between calls.
+ *   - It allocates nothing: no cudaMalloc, no cudaFree, no library allocator.
+ * The paper has no counterpart: this is an interface for such callers only. */
+CMR_API cmr_status cmr_positions_frames_noalloc(const int32_t* ids, const int32_t* cu_seqlens,
+                                                int32_t num_seqs, int64_t n_tokens,
+                                                int32_t image_token_id, int32_t grid_side,
+                                                int32_t* out_pos, int32_t* out_start,
+                                                int32_t* out_amount, int32_t* device_status,
+                                                cmr_stream_t stream);
+
 /* Planes of one new token per sequence, for decode and continuation (port
  * notes: generated tokens sit at p - amount; the canvas table's last row,
  * after the frame, covers generated tokens too).  Token b sits at absolute

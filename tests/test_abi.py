@@ -33,7 +33,8 @@ def test_header_declares_the_entry_points():
                           "cmr_rotate_qk_cache_kernel", "cmr_copy_rotated_dims",
                           "cmr_status_string", "cmr_last_error_message",
                           "cmr_last_rotate_kernel", "cmr_version", "cmr_positions_frames",
-                          "cmr_positions_frames_workspace_bytes"}
+                          "cmr_positions_frames_workspace_bytes",
+                          "cmr_positions_frames_noalloc"}
     assert set(names) == set(cmr.SIGNATURES)
 
 

@@ -36,6 +36,9 @@ SIGNATURES = {
                                             ctypes.c_void_p, ctypes.c_size_t, _i32p,
                                             ctypes.c_void_p]),
     "cmr_positions_frames_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int64]),
+    "cmr_positions_frames_noalloc": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                                    ctypes.c_int32, ctypes.c_int32, _i32p, _i32p,
+                                                    _i32p, _i32p, ctypes.c_void_p]),
     "cmr_positions_step": (ctypes.c_int, [_i32p, _i32p, _i32p, ctypes.c_int32, _i32p,
                                           ctypes.c_void_p]),
     "cmr_rotate_qk_shift": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, _i32p,

@@ -251,6 +251,33 @@ cmr_status cmr_positions_frames(const int32_t* ids, const int32_t* cu_seqlens, i
   return CMR_OK;
 }
 
+cmr_status cmr_positions_frames_noalloc(const int32_t* ids, const int32_t* cu_seqlens,
+                                        int32_t num_seqs, int64_t n_tokens,
+                                        int32_t image_token_id, int32_t grid_side,
+                                        int32_t* out_pos, int32_t* out_start,
+                                        int32_t* out_amount, int32_t* device_status,
+                                        cmr_stream_t stream) {
+  if (grid_side < 1 || grid_side > 128) return fail(CMR_EINVAL, "grid_side must be in 1 .. 128");
+  if (num_seqs > cmr::frames_static_max_seqs())
+    return fail(CMR_EINVAL,
+                "num_seqs = %d exceeds the %lld sequences the built-in scratch serves; "
+                "use cmr_positions_frames with a workspace",
+                num_seqs, static_cast<long long>(cmr::frames_static_max_seqs()));
+  cmr_status s = check_positions(ids, cu_seqlens, num_seqs, n_tokens, out_pos, out_start,
+                                 out_amount, device_status);
+  if (s != CMR_OK || num_seqs == 0) return s;
+  void* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  cudaError_t e = cmr::frames_static_scratch(&scratch, &scratch_bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch");
+  e = cmr::launch_positions_frames(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
+                                   grid_side, out_pos, out_start, out_amount, scratch,
+                                   scratch_bytes, device_status,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "positions_frames_noalloc launch");
+  return CMR_OK;
+}
+
 cmr_status cmr_positions_step(const int32_t* cache_len, const int32_t* start,
                               const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
                               cmr_stream_t stream) {

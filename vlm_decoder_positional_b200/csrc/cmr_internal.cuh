@@ -105,6 +105,12 @@ cudaError_t launch_positions_frames(const int32_t* ids, const int32_t* cu_seqlen
                                     size_t workspace_bytes, int32_t* device_status,
                                     cudaStream_t stream);
 
+// The built-in scratch of cmr_positions_frames_noalloc: its device address on
+// the current device (looked up on the first call per device) and size, and
+// the most sequences it serves (one summary each).
+cudaError_t frames_static_scratch(void** ptr, size_t* bytes);
+int64_t frames_static_max_seqs();
+
 cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start,
                                   const int32_t* amount, int32_t num_seqs, int32_t* out_pos,
                                   cudaStream_t stream);

@@ -27,6 +27,8 @@
 //      and the planes of every token.
 // Ids are read twice (once per kernel; the second read mostly hits L2); the
 // planes are written once.  No CTA waits on another.
+#include <mutex>
+
 #include "canvas.cuh"
 #include "pdl.cuh"
 
@@ -254,6 +256,40 @@ int64_t frames_slices(int32_t num_seqs, int64_t n_tokens, size_t workspace_bytes
 }
 
 size_t frames_summary_bytes() { return sizeof(Summary); }
+
+// ---- built-in scratch for callers that cannot allocate device memory ----
+//
+// cmr_positions_frames_noalloc keeps its slice summaries here instead of in a
+// caller's workspace: kStaticFrameSummaries summaries of 16 bytes (256 KB),
+// held by every device that loads the library until the process exits.  All
+// calls share it, so calls that overlap on the device race; a call writes
+// every summary it reads, so nothing needs clearing between calls.
+constexpr int64_t kStaticFrameSummaries = 16384;
+static __device__ __align__(256) Summary g_frame_scratch[kStaticFrameSummaries];
+
+// The device address of g_frame_scratch on the current device: in host code
+// the array's name stands for a host-side shadow, not device memory, so the
+// address is looked up once per device (with that device current) and cached.
+cudaError_t frames_static_scratch(void** ptr, size_t* bytes) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_frame_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  *bytes = sizeof(g_frame_scratch);
+  return cudaSuccess;
+}
+
+int64_t frames_static_max_seqs() { return kStaticFrameSummaries; }
 
 cudaError_t launch_positions_frames(const int32_t* ids, const int32_t* cu_seqlens,
                                     int32_t num_seqs, int64_t n_tokens, int32_t image_token_id,
