@@ -479,6 +479,10 @@ def run_ours(args):
     # or at its capture into the graph)
     kernel_ran = cmr.last_rotate_kernel() or kernel
 
+    # A step of one call is timed by the two events around the K steps alone
+    # (events recorded between graph launches cost about a microsecond each);
+    # a step of two calls also gets events around each call.
+    single = "positions" not in calls
     rot_events = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3))
                   for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
@@ -489,14 +493,18 @@ def run_ours(args):
     with ClockSampler(local_rank) as clocks:
         t_begin.record(stream)
         for i in range(args.steps):
-            step(rot_events[i])
+            step(None if single else rot_events[i])
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
     ms = t_begin.elapsed_time(t_end)
-    rot_ms = [a.elapsed_time(z) for a, z, _ in rot_events]
-    pos_ms = [p.elapsed_time(a) for a, _, p in rot_events]
+    if single:
+        rot_ms = [ms / args.steps]
+        pos_ms = [0.0]
+    else:
+        rot_ms = [a.elapsed_time(z) for a, z, _ in rot_events]
+        pos_ms = [p.elapsed_time(a) for a, _, p in rot_events]
     ms_max = shard.max_over_ranks(ms, dist, dev)
     # tokens processed by all ranks in one step
     tokens_all = tokens_per_step * world if args.scaling == "weak" else global_tokens
@@ -533,10 +541,11 @@ def run_ours(args):
                     "kernel": kernel_ran,
                     "algorithmic_bytes_per_launch": rot_b,
                     "avg_launch_ms": rot_avg_s * 1e3,
-                    "timed": ("the whole one-call step (CUDA events around it): the positions "
-                              "kernels and the rotation overlapping them, an upper bound of the "
-                              "rotate kernel's own duration" if one_call else
-                              "the rotate launch alone (CUDA events around it)"),
+                    "timed": ("the one-call step (CUDA events around the K steps, divided by "
+                              "K): the origin scan and the rotation overlapping it, an upper "
+                              "bound of the rotate kernel's own duration" if one_call else
+                              "the rotate call alone (events around it)" if not single else
+                              "the rotate call (CUDA events around the K steps, divided by K)"),
                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                     if peak_src == "measured" else "fallback 6650 GB/s",
                     "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS}
@@ -665,8 +674,6 @@ def run_frames(args):
     for _ in range(args.warmup):
         call()
     torch.cuda.synchronize(dev)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if dist:
@@ -674,16 +681,15 @@ def run_frames(args):
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clocks:
         t_begin.record(stream)
-        for a, z in ev:
-            a.record(stream)
+        for _ in range(args.steps):
             call()
-            z.record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
-    ms_max = shard.max_over_ranks(t_begin.elapsed_time(t_end), dist, dev)
-    call_ms = statistics.mean(a.elapsed_time(z) for a, z in ev)
+    ms_local = t_begin.elapsed_time(t_end)
+    ms_max = shard.max_over_ranks(ms_local, dist, dev)
+    call_ms = ms_local / args.steps
     moved = positions_bytes(n, b)
     if rank == 0:
         peak, peak_src = measured_peak()
@@ -725,8 +731,8 @@ def run_frames(args):
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "frames_positions_kernel (+ frames_summary_kernel)",
                          "algorithmic_bytes_per_launch": moved, "avg_launch_ms": call_ms,
-                         "timed": "the whole call (CUDA events around it): the summary and "
-                                  "planes kernels",
+                         "timed": "the call (CUDA events around the K calls, divided by K): "
+                                  "the summary and planes kernels",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6650 GB/s",
                          "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS},

@@ -145,3 +145,30 @@ def test_graph_replay_and_the_rotation_with_frame_planes(cuda_device):
     torch.cuda.synchronize()
     got = q[..., :64].contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
     BarStats("q with frame planes").add(got, oracle_rotate_threads(q_in, want)).check()
+
+
+def test_unaligned_buffers_and_odd_token_counts(cuda_device):
+    # ids and the planes at addresses that are not 16-byte aligned, and token
+    # counts that leave the plane rows unaligned: element-wise paths
+    dev = cuda_device
+    rng = np.random.default_rng(600)
+    for n_extra in (0, 1, 2, 3):
+        ids_np, cu_np = random_batch(rng, 8, 9, 5000)
+        if n_extra:
+            ids_np = np.concatenate([ids_np, inputs.text_ids(rng, n_extra)])
+            cu_np = cu_np.copy()
+            cu_np[-1] += n_extra
+        n, b = ids_np.shape[0], cu_np.shape[0] - 1
+        want = oracle.positions_frames(ids_np, cu_np, MARK, 8)
+        for shift in (0, 1, 3):
+            ids_buf = torch.zeros(n + 4, dtype=torch.int32, device=dev)
+            ids_buf[shift:shift + n] = t32(ids_np, dev)
+            pos_buf = torch.full((3 * n + 4,), -5, dtype=torch.int32, device=dev)
+            pos = pos_buf[shift:shift + 3 * n].view(3, n)
+            st = torch.empty(b, dtype=torch.int32, device=dev)
+            am = torch.empty(b, dtype=torch.int32, device=dev)
+            cmr.positions_frames(ids_buf[shift:shift + n], t32(cu_np, dev), 8, out=(pos, st, am))
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(pos.cpu().numpy(), want[0])
+            np.testing.assert_array_equal(st.cpu().numpy(), want[1])
+            assert (pos_buf[:shift] == -5).all() and (pos_buf[shift + 3 * n:] == -5).all()

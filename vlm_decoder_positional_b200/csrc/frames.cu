@@ -22,11 +22,17 @@
 //      in a caller-provided workspace [num_seqs][slices];
 //   2. frames_positions_kernel, launched programmatically behind it, folds the
 //      summaries of the slices before its own into a carry (slice 0 folds all
-//      of them for the state), then walks its slice in chunks of kFrThreads
-//      tokens: a warp scan by shuffles, a scan of the warp totals, the carry,
-//      and the planes of every token.
-// Ids are read twice (once per kernel; the second read mostly hits L2); the
-// planes are written once.  No CTA waits on another.
+//      of them for the state), then walks its slice in chunks of
+//      kFrThreads x kFrItems tokens: each thread folds its own kFrItems
+//      consecutive tokens, one block scan of the threads' summaries gives
+//      each thread its prefix, and the thread walks its tokens again writing
+//      their planes.
+// Each thread owns 8 consecutive tokens at an 8-aligned index of the packed
+// batch, so ids are read and planes written as 16-byte vectors (plane rows
+// are 16-byte aligned when n_tokens is a multiple of 4; otherwise, and at
+// the edges of a slice, element by element).  Ids are read twice (once per
+// kernel; the second read mostly hits L2); the planes are written once.  No
+// CTA waits on another.
 #include <mutex>
 
 #include "canvas.cuh"
@@ -35,10 +41,11 @@
 namespace cmr {
 namespace {
 
-constexpr int kFrThreads = 512;
+constexpr int kFrThreads = 256;
 constexpr int kFrWarps = kFrThreads / 32;
-constexpr int kFrPerThread = 4;                              // ids in flight per thread
-constexpr int kFrSliceTarget = kFrThreads * kFrPerThread;    // 2048 tokens per CTA
+constexpr int kFrItems = 8;                                  // consecutive tokens per thread
+constexpr int kFrChunk = kFrThreads * kFrItems;              // 2048 tokens per block step
+constexpr int kFrSliceTarget = kFrChunk;                     // tokens per CTA (target)
 constexpr int kFrMaxSlices = 65535;                          // gridDim.y limit
 
 // Prefix summary of a run of tokens: n markers, the first and last of them
@@ -91,6 +98,47 @@ __device__ __forceinline__ Summary block_scan(Summary v, int32_t frame_len, Summ
   return combine(before, v, frame_len);
 }
 
+// Block-wide exclusive scan in thread order (thread 0 gets the identity);
+// *total receives the block's summary.  Same barriers as block_scan.
+__device__ __forceinline__ Summary block_exclusive_scan(Summary v, int32_t frame_len,
+                                                        Summary* s_warp, Summary* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const Summary incl = warp_scan(v, frame_len);
+  Summary excl = shfl_up(incl, 1);
+  if (lane == 0) excl = Summary{0, 0, 0, 0};
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    Summary w = lane < kFrWarps ? s_warp[lane] : Summary{0, 0, 0, 0};
+    w = warp_scan(w, frame_len);
+    if (lane < kFrWarps) s_warp[lane] = w;
+  }
+  __syncthreads();
+  const Summary before = warp > 0 ? s_warp[warp - 1] : Summary{0, 0, 0, 0};
+  *total = s_warp[kFrWarps - 1];
+  __syncthreads();
+  return combine(before, excl, frame_len);
+}
+
+// The kFrItems ids of the 8-aligned group at global index g of the packed
+// batch; entries outside [lo, hi) read as `none`.  Two 16-byte loads when the
+// group lies inside and ids is 16-byte aligned, else one load per id.
+__device__ __forceinline__ void load_group(const int32_t* __restrict__ ids, int64_t g,
+                                           int64_t lo, int64_t hi, int32_t none,
+                                           int32_t (&v)[kFrItems]) {
+  const bool aligned = (reinterpret_cast<uintptr_t>(ids) & 15u) == 0;
+  if (aligned && g >= lo && g + kFrItems <= hi) {
+    const int4 a = __ldg(reinterpret_cast<const int4*>(ids + g));
+    const int4 b = __ldg(reinterpret_cast<const int4*>(ids + g) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kFrItems; ++j)
+      v[j] = (g + j >= lo && g + j < hi) ? __ldg(ids + g + j) : none;
+  }
+}
+
 struct FrSlice {
   int64_t first, len, p0, p1;
 };
@@ -125,23 +173,24 @@ __global__ void __launch_bounds__(kFrThreads)
       atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
     return;
   }
-  const int32_t* __restrict__ seq = ids + sl.first;
+  // the slice as global indices of the packed batch, walked in 8-aligned
+  // groups of kFrItems tokens, kFrChunk tokens per block step
+  const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
   Summary run{0, 0, 0, 0};
-  for (int64_t c = sl.p0; c < sl.p1; c += kFrSliceTarget) {
-    int32_t v[kFrPerThread];
+  for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi; c += kFrChunk) {
+    const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
+    int32_t v[kFrItems];
+    load_group(ids, g, lo, hi, ~marker, v);
+    Summary mine{0, 0, 0, 0};
 #pragma unroll
-    for (int m = 0; m < kFrPerThread; ++m) {
-      const int64_t p = c + m * kFrThreads + threadIdx.x;
-      v[m] = (p < sl.p1) ? __ldg(seq + p) : ~marker;
-    }
-#pragma unroll
-    for (int m = 0; m < kFrPerThread; ++m) {
-      const int32_t p = static_cast<int32_t>(c + m * kFrThreads + threadIdx.x);
-      Summary e = (v[m] == marker) ? Summary{1, p, p, 0} : Summary{0, 0, 0, 0};
-      Summary total;
-      block_scan(e, frame_len, s_warp, &total);
-      run = combine(run, total, frame_len);
-    }
+    for (int j = 0; j < kFrItems; ++j)
+      if (v[j] == marker) {
+        const int32_t p = static_cast<int32_t>(g + j - sl.first);  // local index
+        mine = combine(mine, Summary{1, p, p, 0}, frame_len);
+      }
+    Summary total;
+    block_scan(mine, frame_len, s_warp, &total);
+    run = combine(run, total, frame_len);
   }
   if (threadIdx.x == 0)
     work[static_cast<int64_t>(blockIdx.x) * gridDim.y + blockIdx.y] = run;
@@ -192,53 +241,73 @@ __global__ void __launch_bounds__(kFrThreads)
   }
   Summary carry = fold(sums, blockIdx.y, frame_len, s_warp);
 
-  const int32_t* __restrict__ seq = ids + sl.first;
-  int32_t* __restrict__ pt = pos + sl.first;
-  int32_t* __restrict__ ph = pos + n_tokens + sl.first;
-  int32_t* __restrict__ pw = pos + 2 * n_tokens + sl.first;
+  const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
   const int64_t rows = static_cast<int64_t>(side) * side;
-  for (int64_t c = sl.p0; c < sl.p1; c += kFrSliceTarget) {
-    int32_t v[kFrPerThread];
+  // plane rows start 16-byte aligned when pos is and n_tokens is a multiple of 4
+  const bool vec = (n_tokens & 3) == 0 && (reinterpret_cast<uintptr_t>(pos) & 15u) == 0;
+  for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi; c += kFrChunk) {
+    const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
+    int32_t v[kFrItems];
+    load_group(ids, g, lo, hi, ~marker, v);
+    Summary mine{0, 0, 0, 0};
 #pragma unroll
-    for (int m = 0; m < kFrPerThread; ++m) {
-      const int64_t p = c + m * kFrThreads + threadIdx.x;
-      v[m] = (p < sl.p1) ? __ldg(seq + p) : ~marker;
-    }
+    for (int j = 0; j < kFrItems; ++j)
+      if (v[j] == marker) {
+        const int32_t p = static_cast<int32_t>(g + j - sl.first);
+        mine = combine(mine, Summary{1, p, p, 0}, frame_len);
+      }
+    Summary total;
+    Summary pre = combine(carry, block_exclusive_scan(mine, frame_len, s_warp, &total),
+                          frame_len);
+    carry = combine(carry, total, frame_len);
+    int32_t t[kFrItems], h[kFrItems], w[kFrItems];
 #pragma unroll
-    for (int m = 0; m < kFrPerThread; ++m) {
-      const int64_t p = c + m * kFrThreads + threadIdx.x;
-      const int32_t p32 = static_cast<int32_t>(p);
-      Summary e = (v[m] == marker) ? Summary{1, p32, p32, 0} : Summary{0, 0, 0, 0};
-      Summary total;
-      const Summary incl = combine(carry, block_scan(e, frame_len, s_warp, &total), frame_len);
-      carry = combine(carry, total, frame_len);
-      if (p >= sl.p1) continue;
-      int64_t t, h, w;
-      if (incl.n == 0) {
-        t = h = w = p;
+    for (int j = 0; j < kFrItems; ++j) {
+      const int64_t p = g + j - sl.first;  // local index
+      if (v[j] == marker)
+        pre = combine(pre, Summary{1, static_cast<int32_t>(p), static_cast<int32_t>(p), 0},
+                      frame_len);
+      int64_t pt, ph, pw;
+      if (pre.n == 0) {
+        pt = ph = pw = p;
       } else {
-        const int64_t anchor = incl.first + static_cast<int64_t>(incl.n - 1) * span + incl.gaps;
-        const int64_t d = p - incl.last;  // offset into the last frame opened
+        const int64_t anchor = pre.first + static_cast<int64_t>(pre.n - 1) * span + pre.gaps;
+        const int64_t d = p - pre.last;  // offset into the last frame opened
         if (d == 0) {
-          t = anchor;
-          h = w = anchor - 1;
+          pt = anchor;
+          ph = pw = anchor - 1;
         } else if (d <= rows) {
           const int64_t k = d - 1;
-          t = anchor;
-          h = anchor + k / side;
-          w = anchor + k % side;
+          pt = anchor;
+          ph = anchor + k / side;
+          pw = anchor + k % side;
         } else if (d == rows + 1) {
-          t = anchor;
-          h = w = anchor + side;
+          pt = anchor;
+          ph = pw = anchor + side;
         } else if (d == rows + 2) {
-          t = h = w = anchor;
+          pt = ph = pw = anchor;
         } else {
-          t = h = w = anchor + span + (d - frame_len);
+          pt = ph = pw = anchor + span + (d - frame_len);
         }
       }
-      pt[p] = static_cast<int32_t>(t);
-      ph[p] = static_cast<int32_t>(h);
-      pw[p] = static_cast<int32_t>(w);
+      t[j] = static_cast<int32_t>(pt);
+      h[j] = static_cast<int32_t>(ph);
+      w[j] = static_cast<int32_t>(pw);
+    }
+    int32_t* const planes[3] = {pos + g, pos + n_tokens + g, pos + 2 * n_tokens + g};
+    const int32_t* const vals[3] = {t, h, w};
+    if (vec && g >= lo && g + kFrItems <= hi) {
+#pragma unroll
+      for (int r = 0; r < 3; ++r) {
+        int4* dst = reinterpret_cast<int4*>(planes[r]);
+        dst[0] = make_int4(vals[r][0], vals[r][1], vals[r][2], vals[r][3]);
+        dst[1] = make_int4(vals[r][4], vals[r][5], vals[r][6], vals[r][7]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kFrItems; ++j)
+        if (g + j >= lo && g + j < hi)
+          for (int r = 0; r < 3; ++r) planes[r][j] = vals[r][j];
     }
   }
 }
