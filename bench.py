@@ -45,6 +45,7 @@ SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (DGX figure)
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_staged.cu",
                   "vlm_decoder_positional_b200/csrc/tma.cuh",
+                  "vlm_decoder_positional_b200/csrc/pdl.cuh",
                   "vlm_decoder_positional_b200/csrc/tensor_map.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_common.cuh",
                   "vlm_decoder_positional_b200/csrc/canvas.cuh",
@@ -509,11 +510,11 @@ def run_ours(args):
     # tokens processed by all ranks in one step
     tokens_all = tokens_per_step * world if args.scaling == "weak" else global_tokens
     # kernels per step: the positions form launches two (origin scan, planes),
-    # each rotate form one
+    # each rotate form one, the one-call path two (origin scan, rotation)
     per_step = {"positions": 2, "rotate": 1}
     launches = args.steps * sum(per_step[name] for name, _ in plan)
     if step_kind(args, wl) == "one-call":
-        launches = args.steps * 3
+        launches = args.steps * 2
 
     # end to end through the public API from pinned host memory
     if args.op == "rotate":

@@ -30,7 +30,7 @@ def test_bench_line_keeps_the_contract(launch):
     assert d["n_gpus"] == 1 and d["steps"] == 4 and d["warmup"] == 3
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["scaling"] == "weak" and d["vs_baseline"] is None
-    assert d["gpu_launches"] == 3 * 4   # origin scan + planes + rotation per step
+    assert d["gpu_launches"] == 2 * 4   # origin scan + rotation per step
     assert d["config"]["step"] == "one-call" and d["positions_avg_ms"] is None
     assert "workload" in d["config"]
     r = d["roofline"]

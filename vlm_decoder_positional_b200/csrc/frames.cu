@@ -66,8 +66,10 @@ __device__ __forceinline__ Summary shfl_up(const Summary& v, int delta) {
           __shfl_up_sync(0xffffffffu, v.last, delta), __shfl_up_sync(0xffffffffu, v.gaps, delta)};
 }
 
-// Inclusive scan over the warp's lanes in lane order.
+// Inclusive scan over the warp's lanes in lane order.  A warp holding no
+// marker (the common case: frames are sparse) is all identities already.
 __device__ __forceinline__ Summary warp_scan(Summary v, int32_t frame_len) {
+  if (!__any_sync(0xffffffffu, v.n != 0)) return v;
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -77,47 +79,52 @@ __device__ __forceinline__ Summary warp_scan(Summary v, int32_t frame_len) {
   return v;
 }
 
-// Block-wide inclusive scan in thread order; *total receives the block's
-// summary.  All threads must call it; it uses s_warp[kFrWarps] and two
-// barriers.
-__device__ __forceinline__ Summary block_scan(Summary v, int32_t frame_len, Summary* s_warp,
-                                              Summary* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_scan(v, frame_len);
-  if (lane == 31) s_warp[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    Summary w = lane < kFrWarps ? s_warp[lane] : Summary{0, 0, 0, 0};
-    w = warp_scan(w, frame_len);
-    if (lane < kFrWarps) s_warp[lane] = w;  // inclusive prefix of the warp totals
-  }
-  __syncthreads();
-  const Summary before = warp > 0 ? s_warp[warp - 1] : Summary{0, 0, 0, 0};
-  *total = s_warp[kFrWarps - 1];
-  __syncthreads();  // s_warp is rewritten by the next call
-  return combine(before, v, frame_len);
-}
+// Block-wide scans and reductions in thread order, with one barrier each.
+// Each call takes the next of two shared buffers of warp totals (BlockBufs):
+// two calls in a row never share a buffer, and a call reusing one runs after
+// the barrier of the call between, which every thread passes only once it
+// has read the older call's totals.  All threads must make the same calls.
+struct BlockBufs {
+  Summary warp[2][kFrWarps];
+};
 
-// Block-wide exclusive scan in thread order (thread 0 gets the identity);
-// *total receives the block's summary.  Same barriers as block_scan.
+// Exclusive prefix of v in thread order (thread 0: the identity); *total
+// receives the block's summary.
 __device__ __forceinline__ Summary block_exclusive_scan(Summary v, int32_t frame_len,
-                                                        Summary* s_warp, Summary* total) {
+                                                        BlockBufs& bufs, int& turn,
+                                                        Summary* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Summary* const buf = bufs.warp[turn];
+  turn ^= 1;
   const Summary incl = warp_scan(v, frame_len);
   Summary excl = shfl_up(incl, 1);
   if (lane == 0) excl = Summary{0, 0, 0, 0};
-  if (lane == 31) s_warp[warp] = incl;
+  if (lane == 31) buf[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    Summary w = lane < kFrWarps ? s_warp[lane] : Summary{0, 0, 0, 0};
-    w = warp_scan(w, frame_len);
-    if (lane < kFrWarps) s_warp[lane] = w;
+  Summary before{0, 0, 0, 0}, all{0, 0, 0, 0};
+#pragma unroll
+  for (int w = 0; w < kFrWarps; ++w) {
+    const Summary t = buf[w];
+    if (w < warp) before = combine(before, t, frame_len);
+    all = combine(all, t, frame_len);
   }
-  __syncthreads();
-  const Summary before = warp > 0 ? s_warp[warp - 1] : Summary{0, 0, 0, 0};
-  *total = s_warp[kFrWarps - 1];
-  __syncthreads();
+  *total = all;
   return combine(before, excl, frame_len);
+}
+
+// The block's summary of v in thread order.
+__device__ __forceinline__ Summary block_reduce(Summary v, int32_t frame_len, BlockBufs& bufs,
+                                                int& turn) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Summary* const buf = bufs.warp[turn];
+  turn ^= 1;
+  const Summary incl = warp_scan(v, frame_len);
+  if (lane == 31) buf[warp] = incl;
+  __syncthreads();
+  Summary all{0, 0, 0, 0};
+#pragma unroll
+  for (int w = 0; w < kFrWarps; ++w) all = combine(all, buf[w], frame_len);
+  return all;
 }
 
 // The kFrItems ids of the 8-aligned group at global index g of the packed
@@ -164,7 +171,8 @@ __global__ void __launch_bounds__(kFrThreads)
     frames_summary_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                           int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t frame_len,
                           Summary* __restrict__ work, int32_t* __restrict__ status) {
-  __shared__ Summary s_warp[kFrWarps];
+  __shared__ BlockBufs bufs;
+  int turn = 0;
   pdl::launch_dependents();
   bool bad;
   FrSlice sl;
@@ -188,9 +196,7 @@ __global__ void __launch_bounds__(kFrThreads)
         const int32_t p = static_cast<int32_t>(g + j - sl.first);  // local index
         mine = combine(mine, Summary{1, p, p, 0}, frame_len);
       }
-    Summary total;
-    block_scan(mine, frame_len, s_warp, &total);
-    run = combine(run, total, frame_len);
+    run = combine(run, block_reduce(mine, frame_len, bufs, turn), frame_len);
   }
   if (threadIdx.x == 0)
     work[static_cast<int64_t>(blockIdx.x) * gridDim.y + blockIdx.y] = run;
@@ -198,25 +204,24 @@ __global__ void __launch_bounds__(kFrThreads)
 
 // Ordered fold of summaries[0, count) by the whole block.  The summaries come
 // from the kernel before (plain loads, not the read-only path).
-__device__ __forceinline__ Summary fold(const Summary* sums, int32_t count,
-                                        int32_t frame_len, Summary* s_warp) {
+__device__ __forceinline__ Summary fold(const Summary* sums, int32_t count, int32_t frame_len,
+                                        BlockBufs& bufs, int& turn) {
   Summary acc{0, 0, 0, 0};
   for (int32_t base = 0; base < count; base += kFrThreads) {
     const int32_t j = base + threadIdx.x;
-    Summary e = j < count ? sums[j] : Summary{0, 0, 0, 0};
-    Summary total;
-    block_scan(e, frame_len, s_warp, &total);
-    acc = combine(acc, total, frame_len);
+    const Summary e = j < count ? sums[j] : Summary{0, 0, 0, 0};
+    acc = combine(acc, block_reduce(e, frame_len, bufs, turn), frame_len);
   }
   return acc;
 }
 
-__global__ void __launch_bounds__(kFrThreads)
+__global__ void __launch_bounds__(kFrThreads, 5)
     frames_positions_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                             int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t side,
                             const Summary* work, int32_t* __restrict__ pos,
                             int32_t* __restrict__ out_start, int32_t* __restrict__ out_amount) {
-  __shared__ Summary s_warp[kFrWarps];
+  __shared__ BlockBufs bufs;
+  int turn = 0;
   bool bad;
   FrSlice sl;
   if (!fr_slice(cu, num_seqs, n_tokens, &bad, &sl)) return;
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(kFrThreads)
   const Summary* sums = work + static_cast<int64_t>(blockIdx.x) * gridDim.y;
   pdl::wait();  // the summaries are written
   if (blockIdx.y == 0) {
-    const Summary all = fold(sums, gridDim.y, frame_len, s_warp);
+    const Summary all = fold(sums, gridDim.y, frame_len, bufs, turn);
     if (threadIdx.x == 0) {
       if (all.n == 0) {
         out_start[blockIdx.x] = kTextOnlyStart;
@@ -239,10 +244,14 @@ __global__ void __launch_bounds__(kFrThreads)
       }
     }
   }
-  Summary carry = fold(sums, blockIdx.y, frame_len, s_warp);
+  Summary carry = fold(sums, blockIdx.y, frame_len, bufs, turn);
 
   const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
-  const int64_t rows = static_cast<int64_t>(side) * side;
+  // per-token arithmetic in 32 bits: every coordinate fits in int32 (a
+  // documented limit), and so does every intermediate below
+  const int32_t rows = side * side;
+  const uint32_t uside = static_cast<uint32_t>(side);
+  const int32_t span32 = side + 1;
   // plane rows start 16-byte aligned when pos is and n_tokens is a multiple of 4
   const bool vec = (n_tokens & 3) == 0 && (reinterpret_cast<uintptr_t>(pos) & 15u) == 0;
   for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi; c += kFrChunk) {
@@ -257,42 +266,41 @@ __global__ void __launch_bounds__(kFrThreads)
         mine = combine(mine, Summary{1, p, p, 0}, frame_len);
       }
     Summary total;
-    Summary pre = combine(carry, block_exclusive_scan(mine, frame_len, s_warp, &total),
+    Summary pre = combine(carry, block_exclusive_scan(mine, frame_len, bufs, turn, &total),
                           frame_len);
     carry = combine(carry, total, frame_len);
     int32_t t[kFrItems], h[kFrItems], w[kFrItems];
 #pragma unroll
     for (int j = 0; j < kFrItems; ++j) {
-      const int64_t p = g + j - sl.first;  // local index
-      if (v[j] == marker)
-        pre = combine(pre, Summary{1, static_cast<int32_t>(p), static_cast<int32_t>(p), 0},
-                      frame_len);
-      int64_t pt, ph, pw;
+      const int32_t p = static_cast<int32_t>(g + j - sl.first);  // local index
+      if (v[j] == marker) pre = combine(pre, Summary{1, p, p, 0}, frame_len);
+      int32_t pt, ph, pw;
       if (pre.n == 0) {
         pt = ph = pw = p;
       } else {
-        const int64_t anchor = pre.first + static_cast<int64_t>(pre.n - 1) * span + pre.gaps;
-        const int64_t d = p - pre.last;  // offset into the last frame opened
+        const int32_t anchor = pre.first + (pre.n - 1) * span32 + pre.gaps;
+        const int32_t d = p - pre.last;  // offset into the last frame opened
         if (d == 0) {
           pt = anchor;
           ph = pw = anchor - 1;
         } else if (d <= rows) {
-          const int64_t k = d - 1;
+          const uint32_t k = static_cast<uint32_t>(d - 1);
+          const uint32_t q = k / uside;
           pt = anchor;
-          ph = anchor + k / side;
-          pw = anchor + k % side;
+          ph = anchor + static_cast<int32_t>(q);
+          pw = anchor + static_cast<int32_t>(k - q * uside);
         } else if (d == rows + 1) {
           pt = anchor;
           ph = pw = anchor + side;
         } else if (d == rows + 2) {
           pt = ph = pw = anchor;
         } else {
-          pt = ph = pw = anchor + span + (d - frame_len);
+          pt = ph = pw = anchor + span32 + (d - frame_len);
         }
       }
-      t[j] = static_cast<int32_t>(pt);
-      h[j] = static_cast<int32_t>(ph);
-      w[j] = static_cast<int32_t>(pw);
+      t[j] = pt;
+      h[j] = ph;
+      w[j] = pw;
     }
     int32_t* const planes[3] = {pos + g, pos + n_tokens + g, pos + 2 * n_tokens + g};
     const int32_t* const vals[3] = {t, h, w};
