@@ -636,6 +636,72 @@ def run_probe_only(args):
     return 0
 
 
+def frames_config(args, wl, world):
+    n, b = wl.n_tokens, wl.num_seqs
+    return {"workload": f"{wl.name}: {b} prompts x {n // b} tokens, "
+                        f"{args.frames_per_prompt} frames each, grid side {args.grid_side}",
+            "global_batch": n * world, "launch": args.launch, "op": "frames",
+            "step": "separate", "seq_len": n // b,
+            "parallelism": f"dp{world} (independent batches, no data-path collective)",
+            "l2": "inputs larger than L2 (%.0f MB of ids and planes per step, L2 126 MB); no "
+                  "flush" % (positions_bytes(n, b) / 1e6)}
+
+
+def run_frames_reference(args):
+    """--impl reference --op frames: the oracle's multi-frame planes on all
+    host cores (whole prompts split over a thread pool), on a bounded sample
+    of the multi-frame workload per step."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    wl = inputs.make_frames_workload(frames=args.frames_per_prompt, grid_side=args.grid_side)
+    cores = host_cores()
+    cu = wl.cu_seqlens
+
+    def run(take):
+        cuts = np.linspace(0, take, cores + 1).astype(int)
+
+        def part(i):
+            lo, hi = cuts[i], cuts[i + 1]
+            if hi > lo:
+                oracle.positions_frames(wl.ids[cu[lo]:cu[hi]], cu[lo:hi + 1] - cu[lo],
+                                        wl.image_token_id, args.grid_side)
+        with ThreadPoolExecutor(cores) as ex:
+            list(ex.map(part, range(cores)))
+
+    per_step = max(0.5, args.reference_budget_s / (args.steps + args.warmup))
+    take = 1
+    while take < wl.num_seqs:
+        t0 = time.perf_counter()
+        run(take)
+        if time.perf_counter() - t0 > per_step / 2:
+            break
+        take = min(wl.num_seqs, take * 2)
+    for _ in range(args.warmup):
+        run(take)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run(take)
+    dt = time.perf_counter() - t0
+    n = int(cu[take])
+    value = n * args.steps / dt
+    sample = (f"per step: multi-frame planes of the first {take} prompts ({n} tokens), "
+              f"the oracle (integer arithmetic) on {cores} host threads")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int32", "data": "synthetic (seeded)",
+        "config": frames_config(args, wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }), flush=True)
+    return 0
+
+
 def run_frames(args):
     """--op frames: one step = cmr_positions_frames (multi-frame canvas planes)
     on the multi-frame workload (256 prompts x 65,536 tokens, 32 frames each,
@@ -720,14 +786,7 @@ def run_frames(args):
             "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int32",
             "data": "synthetic (seeded uniform text ids, frames on a grid_side x grid_side grid)",
-            "config": {"workload": f"{wl.name}: {b} prompts x {n // b} tokens, "
-                                   f"{args.frames_per_prompt} frames each, grid side "
-                                   f"{args.grid_side}", "global_batch": tokens_all,
-                       "launch": args.launch, "op": "frames", "step": "separate",
-                       "seq_len": n // b, "parallelism": f"dp{world} (independent batches, no "
-                                                         "data-path collective)",
-                       "l2": "inputs larger than L2 (%.0f MB of ids and planes per step, L2 "
-                             "126 MB); no flush" % (moved / 1e6)},
+            "config": frames_config(args, wl, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "frames_positions_kernel (+ frames_summary_kernel)",
@@ -871,7 +930,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
-        return run_reference(args)
+        return run_frames_reference(args) if args.op == "frames" else run_reference(args)
     if args.probe:
         return run_probe_only(args)
     if args.op == "frames":

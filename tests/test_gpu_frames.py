@@ -1,8 +1,8 @@
 """GPU parity of the multi-frame canvas (cmr_positions_frames) with the
 oracle, bit for bit: grid sides 1 .. 16, several frames per prompt (spaced,
 crowded, cut short, truncated), text-only and empty prompts, prompts spanning
-many slices, reduced workspaces, a CUDA-graph replay, and the rotation with
-the planes it writes."""
+many slices, reduced and stale workspaces, a CUDA-graph replay, unaligned buffers, the rotation with the
+planes it writes, and decode after the last frame."""
 import numpy as np
 import pytest
 import torch
@@ -95,6 +95,7 @@ def test_small_workspaces_give_the_same_planes(cuda_device):
     for nbytes in (16 * b, 16 * b + 15, 32 * b, full - 16, full, full + 4096):
         ws = torch.full((nbytes,), 0x5A, dtype=torch.uint8, device=dev)  # stale contents
         run_both(ids, cu, dev, 8, workspace=ws)
+        run_both(ids, cu, dev, 8, workspace=ws)  # and what the previous call left
     with pytest.raises(cmr.CmrError):
         cmr.positions_frames(t32(ids, dev), t32(cu, dev), 8,
                              workspace=torch.empty(16 * b - 1, dtype=torch.uint8, device=dev))
@@ -172,3 +173,41 @@ def test_unaligned_buffers_and_odd_token_counts(cuda_device):
             np.testing.assert_array_equal(pos.cpu().numpy(), want[0])
             np.testing.assert_array_equal(st.cpu().numpy(), want[1])
             assert (pos_buf[:shift] == -5).all() and (pos_buf[shift + 3 * n:] == -5).all()
+
+
+def test_decode_continues_after_the_last_frame(cuda_device):
+    # the state of a multi-frame prompt drives the decode forms: the planes of
+    # each later token (cmr_positions_step, and the rotation deriving them in
+    # the kernel) equal the oracle's on the prompt extended with text
+    dev = cuda_device
+    rng = np.random.default_rng(700)
+    for s in (2, 8, 16):
+        F = s * s + 3
+        prompts, longer = [], []
+        for i in range(6):
+            count = int(rng.integers(0, 4))
+            origins = inputs.spaced_origins(rng, count, 0, count * (F + 40), F + 1) if count else []
+            full = inputs.prompt_ids_frames(rng, (origins[-1] if origins else 0) + F + 60,
+                                            origins, s)
+            cut = (origins[-1] + F if origins else 0) + int(rng.integers(0, 20))
+            prompts.append(full[:cut])
+            longer.append(full)
+        ids_np, cu_np = inputs.pack(prompts)
+        _, start, amount = cmr.positions_frames(t32(ids_np, dev), t32(cu_np, dev), s)
+        cache_len = np.array([p.shape[0] for p in prompts], np.int32)
+        got = cmr.positions_step(t32(cache_len, dev), start, amount).cpu().numpy()
+        for b, full in enumerate(longer):
+            want, _, _ = oracle.positions_frames(*(np.asarray(full, np.int32),
+                                                   np.array([0, full.shape[0]], np.int32)),
+                                                 MARK, s)
+            np.testing.assert_array_equal(got[:, b], want[:, cache_len[b]])
+        # the same planes, derived inside the rotation (one token per sequence)
+        n = len(prompts)
+        q = inputs.random_qk((1, n, 8, 256), 70 + s, dev)
+        k = inputs.random_qk((1, n, 2, 256), 80 + s, dev)
+        q2, k2 = q.clone(), k.clone()
+        cmr.rotate_qk_shift(q, k, start, amount, pos_offset=t32(cache_len, dev))
+        cmr.rotate_qk(q2, k2, t32(got, dev))
+        torch.cuda.synchronize()
+        assert torch.equal(q.view(torch.int16), q2.view(torch.int16))
+        assert torch.equal(k.view(torch.int16), k2.view(torch.int16))
