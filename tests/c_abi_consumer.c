@@ -4,7 +4,9 @@
  *                         checks; never touches a GPU
  *   ./consumer device  -- the planes of one 80-token prompt with <image> at
  *                         index 6, in cudaMalloc'd buffers; prints "p T H W"
- *                         lines and "start amount" for the test to compare */
+ *                         lines and "start amount" for the test to compare,
+ *                         then "frames same" if the multi-frame entry point
+ *                         without a workspace gives the same planes */
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -43,6 +45,18 @@ static int host_checks(void) {
   CHECK(strcmp(cmr_rotate_qk_cache_kernel(262144, 6, 8, 2, 256, 64),
                "rotate_qk_cache_staged_kernel") == 0);
   CHECK(cmr_rotate_qk_kernel(0, 6, 8, 2, 256, 64) == NULL);
+  CHECK(strcmp(cmr_last_rotate_kernel(), "") == 0); /* nothing launched yet */
+  /* the one-call path: nothing to do, and its rotate arguments are checked */
+  CHECK(cmr_positions_rotate_qk(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL, 1, 8, 2,
+                                256, 1e7, sections, 64, NULL, NULL) == CMR_OK);
+  CHECK(cmr_positions_rotate_qk(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL, 1, 8, 2,
+                                256, 1e7, bad_sections, 64, NULL, NULL) == CMR_EINVAL);
+  /* several frames per prompt: the workspace size and the host checks */
+  CHECK(cmr_positions_frames_workspace_bytes(32, 32 * 8192) == 16u * 32 * 4);
+  CHECK(cmr_positions_frames(fake, fake, 1, 10, 248078, 0, fake, fake, fake, fake, 1 << 20, NULL,
+                             NULL) == CMR_EINVAL);
+  CHECK(cmr_positions_frames_noalloc(fake, fake, 16385, 16385, 248078, 8, fake, fake, fake, NULL,
+                                     NULL) == CMR_EINVAL);
   printf("host ok\n");
   return 0;
 }
@@ -83,6 +97,20 @@ static int device_run(void) {
   CHECK(cudaMemcpy(&amount, d_amount, sizeof amount, 2) == 0);
   for (int p = 0; p < N; ++p) printf("%d %d %d %d\n", p, pos[p], pos[N + p], pos[2 * N + p]);
   printf("%d %d\n", start, amount);
+  /* one frame at grid side 8 through the entry point that allocates nothing */
+  int32_t* d_pos2;
+  CHECK(cudaMalloc((void**)&d_pos2, 3 * N * sizeof(int32_t)) == 0);
+  s = cmr_positions_frames_noalloc(d_ids, d_cu, 1, N, 248078, 8, d_pos2, d_start, d_amount, NULL,
+                                   NULL);
+  if (s != CMR_OK) {
+    fprintf(stderr, "cmr_positions_frames_noalloc: %s\n", cmr_last_error_message());
+    return 1;
+  }
+  CHECK(cudaDeviceSynchronize() == 0);
+  int32_t pos2[3 * N];
+  CHECK(cudaMemcpy(pos2, d_pos2, sizeof pos2, 2) == 0);
+  if (memcmp(pos, pos2, sizeof pos) == 0) printf("frames same\n");
+  cudaFree(d_pos2);
   cudaFree(d_ids);
   cudaFree(d_cu);
   cudaFree(d_pos);

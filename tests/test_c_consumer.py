@@ -1,6 +1,7 @@
 """A plain C11 program uses the C ABI directly: the header compiles as C with
 -Wall -Werror, the host checks answer without a GPU, and on a GPU the planes
-of the 80-token prompt with <image> at 6 equal the golden table."""
+of the 80-token prompt with <image> at 6 equal the golden table, also through
+the multi-frame entry point that allocates nothing."""
 import os
 import subprocess
 
@@ -40,3 +41,4 @@ def test_c_consumer_device_planes(consumer):
     want = [[int(v) for v in r] for r in golden_rows("canvas_O6_80.txt")]
     assert got == want
     assert lines[80].split() == ["73", "58"]
+    assert lines[81] == "frames same"

@@ -1,5 +1,5 @@
 """GPU parity of the multi-frame canvas (cmr_positions_frames) with the
-oracle, bit for bit: grid sides 1 .. 16, several frames per prompt (spaced,
+oracle, bit for bit: grid sides 1 .. 128, several frames per prompt (spaced,
 crowded, cut short, truncated), text-only and empty prompts, prompts spanning
 many slices, reduced and stale workspaces, a CUDA-graph replay, unaligned buffers, the rotation with the
 planes it writes, and decode after the last frame."""
@@ -58,6 +58,15 @@ def test_random_batches_match_the_oracle(cuda_device, s):
     for crowded in (False, True):
         ids, cu = random_batch(rng, s, 40, 6000, crowded)
         run_both(ids, cu, cuda_device, s)
+
+
+@pytest.mark.parametrize("s", [5, 7, 100, 128])
+def test_other_grid_sides_up_to_the_largest(cuda_device, s):
+    # grid rows k / s for sides that are not powers of two, up to s = 128
+    # (frames of 16,387 tokens), whole and cut short
+    rng = np.random.default_rng(800 + s)
+    ids, cu = random_batch(rng, s, 12, 3 * (s * s + 3) + 500)
+    run_both(ids, cu, cuda_device, s)
 
 
 def test_one_frame_at_s8_equals_cmr_positions(cuda_device):

@@ -16,23 +16,30 @@
 //   f_i = O_0 + i (s + 1) + sum_{j < i} max(0, O_{j+1} - O_j - (s*s + 3)),
 // so token p needs only the inclusive prefix, over the tokens up to p, of
 // (marker count, first marker, last marker, summed excess gaps) -- an
-// associative (not commutative) combine.  Two kernels over CTAs (b, s), one
-// per slice s of prompt b:
-//   1. frames_summary_kernel reduces its slice's tokens to that 16-byte summary
-//      in a caller-provided workspace [num_seqs][slices];
-//   2. frames_positions_kernel, launched programmatically behind it, folds the
-//      summaries of the slices before its own into a carry (slice 0 folds all
-//      of them for the state), then walks its slice in chunks of
-//      kFrThreads x kFrItems tokens: each thread folds its own kFrItems
-//      consecutive tokens, one block scan of the threads' summaries gives
-//      each thread its prefix, and the thread walks its tokens again writing
-//      their planes.
+// associative (not commutative) combine.  Each prompt b is cut into slices
+// of about 2,048 tokens, and two kernels run over them:
+//   1. frames_summary_kernel, CTAs (b, group of kFrSumSlices slices), reduces
+//      each slice's tokens to that 16-byte summary in a caller-provided
+//      workspace [num_seqs][slices]; the first ids of all its slices are in
+//      flight before it folds any;
+//   2. frames_positions_kernel, CTAs (b, slice), launched programmatically
+//      behind it, loads its first ids before it waits for the summaries, has
+//      one warp fold the summaries of the slices before its own into a carry,
+//      then walks its slice in chunks of kFrThreads x kFrItems tokens: each
+//      thread folds its own kFrItems consecutive tokens, one block scan of
+//      the threads' summaries gives each thread its prefix, and the thread
+//      walks its tokens again writing their planes.  The CTA holding the
+//      prompt's last token ends with the whole prompt's summary and writes
+//      its state.
 // Each thread owns 8 consecutive tokens at an 8-aligned index of the packed
-// batch, so ids are read and planes written as 16-byte vectors (plane rows
-// are 16-byte aligned when n_tokens is a multiple of 4; otherwise, and at
-// the edges of a slice, element by element).  Ids are read twice (once per
-// kernel; the second read mostly hits L2); the planes are written once.  No
-// CTA waits on another.
+// batch, so ids are read as 16-byte vectors and each plane row is written in
+// the widest stores its alignment allows (16 bytes when n_tokens is a
+// multiple of 4, 8 when it is even; element by element at the edges of a
+// slice).  A thread whose tokens are all text after a frame (or before the
+// first) writes p + offset on every plane without the per-token cases.  Ids
+// are read twice, once per kernel; the plane stores and the second reads are
+// evict-first, so the second read finds the ids in L2 where it can.  No CTA
+// waits on another.
 #include <mutex>
 
 #include "canvas.cuh"
@@ -47,6 +54,8 @@ constexpr int kFrItems = 8;                                  // consecutive toke
 constexpr int kFrChunk = kFrThreads * kFrItems;              // 2048 tokens per block step
 constexpr int kFrSliceTarget = kFrChunk;                     // tokens per CTA (target)
 constexpr int kFrMaxSlices = 65535;                          // gridDim.y limit
+constexpr int kFrSumSlices = 4;                              // slices per summary CTA
+constexpr int kFrPosBlocks = 5;                              // positions CTAs per SM
 
 // Prefix summary of a run of tokens: n markers, the first and last of them
 // (local indices), and the sum over consecutive marker pairs of the text
@@ -100,7 +109,11 @@ __device__ __forceinline__ Summary block_exclusive_scan(Summary v, int32_t frame
   Summary excl = shfl_up(incl, 1);
   if (lane == 0) excl = Summary{0, 0, 0, 0};
   if (lane == 31) buf[warp] = incl;
-  __syncthreads();
+  // a block without a marker (the common case) has identities everywhere
+  if (!__syncthreads_or(v.n != 0)) {
+    *total = Summary{0, 0, 0, 0};
+    return excl;
+  }
   Summary before{0, 0, 0, 0}, all{0, 0, 0, 0};
 #pragma unroll
   for (int w = 0; w < kFrWarps; ++w) {
@@ -120,7 +133,7 @@ __device__ __forceinline__ Summary block_reduce(Summary v, int32_t frame_len, Bl
   turn ^= 1;
   const Summary incl = warp_scan(v, frame_len);
   if (lane == 31) buf[warp] = incl;
-  __syncthreads();
+  if (!__syncthreads_or(v.n != 0)) return Summary{0, 0, 0, 0};
   Summary all{0, 0, 0, 0};
 #pragma unroll
   for (int w = 0; w < kFrWarps; ++w) all = combine(all, buf[w], frame_len);
@@ -129,193 +142,299 @@ __device__ __forceinline__ Summary block_reduce(Summary v, int32_t frame_len, Bl
 
 // The kFrItems ids of the 8-aligned group at global index g of the packed
 // batch; entries outside [lo, hi) read as `none`.  Two 16-byte loads when the
-// group lies inside and ids is 16-byte aligned, else one load per id.
+// group lies inside and ids is 16-byte aligned, else one load per id.  The
+// summary kernel's loads keep normal L2 priority, so that the ids are still in
+// L2 for the positions kernel's loads, the last of the call, which mark them
+// evict-first (kLast).
+template <bool kLast>
+__device__ __forceinline__ int4 ld_ids4(const int32_t* p) {
+  return kLast ? __ldcs(reinterpret_cast<const int4*>(p)) : __ldg(reinterpret_cast<const int4*>(p));
+}
+template <bool kLast>
+__device__ __forceinline__ int32_t ld_id(const int32_t* p) {
+  return kLast ? __ldcs(p) : __ldg(p);
+}
+
+template <bool kLast>
 __device__ __forceinline__ void load_group(const int32_t* __restrict__ ids, int64_t g,
                                            int64_t lo, int64_t hi, int32_t none,
                                            int32_t (&v)[kFrItems]) {
   const bool aligned = (reinterpret_cast<uintptr_t>(ids) & 15u) == 0;
   if (aligned && g >= lo && g + kFrItems <= hi) {
-    const int4 a = __ldg(reinterpret_cast<const int4*>(ids + g));
-    const int4 b = __ldg(reinterpret_cast<const int4*>(ids + g) + 1);
+    const int4 a = ld_ids4<kLast>(ids + g);
+    const int4 b = ld_ids4<kLast>(ids + g + 4);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else {
 #pragma unroll
     for (int j = 0; j < kFrItems; ++j)
-      v[j] = (g + j >= lo && g + j < hi) ? __ldg(ids + g + j) : none;
+      v[j] = (g + j >= lo && g + j < hi) ? ld_id<kLast>(ids + g + j) : none;
   }
 }
 
+// A prompt's tokens [first, first + len) of the packed batch and the local
+// range [p0, p1) of one of its slices (a prompt's length fits int32).
 struct FrSlice {
-  int64_t first, len, p0, p1;
+  int64_t first;
+  int32_t len, p0, p1;
 };
 
-__device__ __forceinline__ bool fr_slice(const int32_t* __restrict__ cu, int32_t num_seqs,
-                                         int64_t n_tokens, bool* bad, FrSlice* sl) {
+// Prompt blockIdx.x of the batch: false (and *bad set) when its cu_seqlens
+// entries are malformed.
+__device__ __forceinline__ bool fr_prompt(const int32_t* __restrict__ cu, int32_t num_seqs,
+                                          int64_t n_tokens, bool* bad, FrSlice* sl) {
   const int32_t b = blockIdx.x;
   const int64_t first = __ldg(cu + b);
   const int64_t last = __ldg(cu + b + 1);
   *bad = first < 0 || last < first || last > n_tokens || (b == 0 && first != 0) ||
          (b == num_seqs - 1 && last != n_tokens);
   if (*bad) return false;
-  const int64_t len = last - first;
-  const int64_t per = (len + gridDim.y - 1) / gridDim.y;
   sl->first = first;
-  sl->len = len;
-  sl->p0 = min(len, static_cast<int64_t>(blockIdx.y) * per);
-  sl->p1 = min(len, sl->p0 + per);
+  sl->len = static_cast<int32_t>(last - first);
   return true;
+}
+
+// Slice y of `slices` of the prompt: local tokens [p0, p1), ceil(len / slices)
+// per slice (the last ones may be empty).
+__device__ __forceinline__ void fr_range(uint32_t y, uint32_t slices, FrSlice* sl) {
+  const uint32_t len = static_cast<uint32_t>(sl->len);
+  const uint32_t per = len / slices + (len % slices != 0);
+  const uint64_t p0 = static_cast<uint64_t>(y) * per;
+  sl->p0 = static_cast<int32_t>(p0 < len ? p0 : len);
+  sl->p1 = static_cast<int32_t>(min(len, static_cast<uint32_t>(sl->p0) + per));
+}
+
+// The summary of the marker tokens among v (local indices from p_base).
+__device__ __forceinline__ Summary fold_group(const int32_t (&v)[kFrItems], int32_t p_base,
+                                              int32_t marker, int32_t frame_len) {
+  Summary mine{0, 0, 0, 0};
+#pragma unroll
+  for (int j = 0; j < kFrItems; ++j)
+    if (v[j] == marker) mine = combine(mine, Summary{1, p_base + j, p_base + j, 0}, frame_len);
+  return mine;
 }
 
 __global__ void __launch_bounds__(kFrThreads)
     frames_summary_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                           int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t frame_len,
-                          Summary* __restrict__ work, int32_t* __restrict__ status) {
+                          int32_t slices, Summary* __restrict__ work,
+                          int32_t* __restrict__ status) {
   __shared__ BlockBufs bufs;
   int turn = 0;
   pdl::launch_dependents();
   bool bad;
   FrSlice sl;
-  if (!fr_slice(cu, num_seqs, n_tokens, &bad, &sl)) {
+  if (!fr_prompt(cu, num_seqs, n_tokens, &bad, &sl)) {
     if (bad && blockIdx.y == 0 && threadIdx.x == 0 && status != nullptr)
       atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
     return;
   }
-  // the slice as global indices of the packed batch, walked in 8-aligned
-  // groups of kFrItems tokens, kFrChunk tokens per block step
-  const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
-  Summary run{0, 0, 0, 0};
-  for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi; c += kFrChunk) {
-    const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
-    int32_t v[kFrItems];
-    load_group(ids, g, lo, hi, ~marker, v);
-    Summary mine{0, 0, 0, 0};
+  // this CTA's slices y0 .. y0 + kFrSumSlices - 1, each walked in 8-aligned
+  // groups of kFrItems tokens (global indices of the packed batch), kFrChunk
+  // tokens per block step; the first group of every slice is loaded before
+  // any is folded
+  const uint32_t y0 = blockIdx.y * kFrSumSlices;
+  int32_t v[kFrSumSlices][kFrItems];
+  int64_t lo[kFrSumSlices], hi[kFrSumSlices];
 #pragma unroll
-    for (int j = 0; j < kFrItems; ++j)
-      if (v[j] == marker) {
-        const int32_t p = static_cast<int32_t>(g + j - sl.first);  // local index
-        mine = combine(mine, Summary{1, p, p, 0}, frame_len);
-      }
-    run = combine(run, block_reduce(mine, frame_len, bufs, turn), frame_len);
+  for (int r = 0; r < kFrSumSlices; ++r) {
+    fr_range(y0 + r, static_cast<uint32_t>(slices), &sl);
+    lo[r] = sl.first + sl.p0;
+    hi[r] = y0 + r < static_cast<uint32_t>(slices) ? sl.first + sl.p1 : lo[r];
+    const int64_t c = lo[r] & ~static_cast<int64_t>(kFrItems - 1);
+    load_group<false>(ids, c + static_cast<int64_t>(threadIdx.x) * kFrItems, lo[r], hi[r],
+                      ~marker, v[r]);
   }
-  if (threadIdx.x == 0)
-    work[static_cast<int64_t>(blockIdx.x) * gridDim.y + blockIdx.y] = run;
+#pragma unroll
+  for (int r = 0; r < kFrSumSlices; ++r) {
+    if (y0 + r >= static_cast<uint32_t>(slices)) break;  // the same for every thread
+    Summary run{0, 0, 0, 0};
+    for (int64_t c = lo[r] & ~static_cast<int64_t>(kFrItems - 1); c < hi[r]; c += kFrChunk) {
+      const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
+      if (c != (lo[r] & ~static_cast<int64_t>(kFrItems - 1)))
+        load_group<false>(ids, g, lo[r], hi[r], ~marker, v[r]);
+      const Summary mine =
+          fold_group(v[r], static_cast<int32_t>(g - sl.first), marker, frame_len);
+      run = combine(run, block_reduce(mine, frame_len, bufs, turn), frame_len);
+    }
+    if (threadIdx.x == 0) work[static_cast<int64_t>(blockIdx.x) * slices + y0 + r] = run;
+  }
 }
 
-// Ordered fold of summaries[0, count) by the whole block.  The summaries come
-// from the kernel before (plain loads, not the read-only path).
-__device__ __forceinline__ Summary fold(const Summary* sums, int32_t count, int32_t frame_len,
-                                        BlockBufs& bufs, int& turn) {
+// Ordered fold of summaries[0, count) by one warp (all 32 lanes call it);
+// every lane receives the result.  The summaries come from the kernel before
+// (plain loads, not the read-only path).
+__device__ __forceinline__ Summary warp_fold(const Summary* sums, int32_t count,
+                                             int32_t frame_len) {
+  const int lane = threadIdx.x & 31;
   Summary acc{0, 0, 0, 0};
-  for (int32_t base = 0; base < count; base += kFrThreads) {
-    const int32_t j = base + threadIdx.x;
-    const Summary e = j < count ? sums[j] : Summary{0, 0, 0, 0};
-    acc = combine(acc, block_reduce(e, frame_len, bufs, turn), frame_len);
+  for (int32_t base = 0; base < count; base += 32) {
+    const int32_t j = base + lane;
+    Summary e = j < count ? sums[j] : Summary{0, 0, 0, 0};
+    e = warp_scan(e, frame_len);
+    const Summary all = {__shfl_sync(0xffffffffu, e.n, 31), __shfl_sync(0xffffffffu, e.first, 31),
+                         __shfl_sync(0xffffffffu, e.last, 31),
+                         __shfl_sync(0xffffffffu, e.gaps, 31)};
+    acc = combine(acc, all, frame_len);
   }
   return acc;
 }
 
-__global__ void __launch_bounds__(kFrThreads, 5)
+// Four consecutive plane values at dst, in the widest stores dst's alignment
+// allows (16, 8 or 4 bytes; the same for every thread of a plane row, whose
+// groups start at multiples of 8 tokens).  The planes are written once and
+// not read back here: evict-first stores, which leave the ids in L2 for the
+// positions kernel's second read.
+__device__ __forceinline__ void store4(int32_t* dst, int32_t a, int32_t b, int32_t c, int32_t d) {
+  const uintptr_t al = reinterpret_cast<uintptr_t>(dst);
+  if ((al & 15u) == 0) {
+    __stcs(reinterpret_cast<int4*>(dst), make_int4(a, b, c, d));
+  } else if ((al & 7u) == 0) {
+    __stcs(reinterpret_cast<int2*>(dst), make_int2(a, b));
+    __stcs(reinterpret_cast<int2*>(dst) + 1, make_int2(c, d));
+  } else {
+    __stcs(dst, a);
+    __stcs(dst + 1, b);
+    __stcs(dst + 2, c);
+    __stcs(dst + 3, d);
+  }
+}
+
+__global__ void __launch_bounds__(kFrThreads, kFrPosBlocks)
     frames_positions_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                             int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t side,
-                            const Summary* work, int32_t* __restrict__ pos,
+                            uint32_t side_magic, const Summary* work, int32_t* __restrict__ pos,
                             int32_t* __restrict__ out_start, int32_t* __restrict__ out_amount) {
   __shared__ BlockBufs bufs;
+  __shared__ Summary s_carry;
   int turn = 0;
   bool bad;
   FrSlice sl;
-  if (!fr_slice(cu, num_seqs, n_tokens, &bad, &sl)) return;
-  if (blockIdx.y != 0 && sl.p0 >= sl.p1) return;
+  if (!fr_prompt(cu, num_seqs, n_tokens, &bad, &sl)) return;
+  fr_range(blockIdx.y, gridDim.y, &sl);
+  // The CTA holding the prompt's last token (slice 0 of an empty prompt)
+  // ends with the summary of the whole prompt and writes its state.
+  const bool writer = sl.len == 0 ? blockIdx.y == 0 : (sl.p0 < sl.p1 && sl.p1 == sl.len);
+  if (sl.p0 >= sl.p1 && !writer) return;
   const int32_t frame_len = side * side + 3;
-  const int64_t span = side + 1;  // counter advance per frame
-  const Summary* sums = work + static_cast<int64_t>(blockIdx.x) * gridDim.y;
-  pdl::wait();  // the summaries are written
-  if (blockIdx.y == 0) {
-    const Summary all = fold(sums, gridDim.y, frame_len, bufs, turn);
-    if (threadIdx.x == 0) {
-      if (all.n == 0) {
-        out_start[blockIdx.x] = kTextOnlyStart;
-        out_amount[blockIdx.x] = 0;
-      } else {
-        const int64_t start = static_cast<int64_t>(all.last) + frame_len;
-        const int64_t anchor = all.first + static_cast<int64_t>(all.n - 1) * span + all.gaps;
-        out_start[blockIdx.x] = static_cast<int32_t>(start);
-        out_amount[blockIdx.x] = static_cast<int32_t>(start - (anchor + span));
-      }
-    }
-  }
-  Summary carry = fold(sums, blockIdx.y, frame_len, bufs, turn);
-
   const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
+  const int64_t c0 = lo & ~static_cast<int64_t>(kFrItems - 1);
+  // The first group of ids is an input that the summary kernel never writes:
+  // it is loaded before the wait, so its latency overlaps that kernel's tail.
+  int32_t v[kFrItems];
+  if (c0 < hi)
+    load_group<true>(ids, c0 + static_cast<int64_t>(threadIdx.x) * kFrItems, lo, hi, ~marker, v);
+  pdl::wait();  // the summaries are written
+  // warp 0 folds the summaries of the slices before this one; the other
+  // warps read the carry after the first block scan's barrier
+  if (threadIdx.x < 32) {
+    const Summary before =
+        warp_fold(work + static_cast<int64_t>(blockIdx.x) * gridDim.y, blockIdx.y, frame_len);
+    if (threadIdx.x == 0) s_carry = before;
+  }
+  Summary carry{0, 0, 0, 0};  // the prompt's summary up to the current chunk
+
   // per-token arithmetic in 32 bits: every coordinate fits in int32 (a
   // documented limit), and so does every intermediate below
   const int32_t rows = side * side;
-  const uint32_t uside = static_cast<uint32_t>(side);
-  const int32_t span32 = side + 1;
-  // plane rows start 16-byte aligned when pos is and n_tokens is a multiple of 4
-  const bool vec = (n_tokens & 3) == 0 && (reinterpret_cast<uintptr_t>(pos) & 15u) == 0;
-  for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi; c += kFrChunk) {
+  const int32_t span32 = side + 1;  // counter advance per frame
+  for (int64_t c = c0; c < hi; c += kFrChunk) {
     const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
-    int32_t v[kFrItems];
-    load_group(ids, g, lo, hi, ~marker, v);
-    Summary mine{0, 0, 0, 0};
-#pragma unroll
-    for (int j = 0; j < kFrItems; ++j)
-      if (v[j] == marker) {
-        const int32_t p = static_cast<int32_t>(g + j - sl.first);
-        mine = combine(mine, Summary{1, p, p, 0}, frame_len);
-      }
+    if (c != c0) load_group<true>(ids, g, lo, hi, ~marker, v);
+    const int32_t p_base = static_cast<int32_t>(g - sl.first);  // local index of v[0]
+    const Summary mine = fold_group(v, p_base, marker, frame_len);
     Summary total;
-    Summary pre = combine(carry, block_exclusive_scan(mine, frame_len, bufs, turn, &total),
-                          frame_len);
+    const Summary excl = block_exclusive_scan(mine, frame_len, bufs, turn, &total);
+    if (c == c0) carry = s_carry;  // written before that scan's barrier
+    Summary pre = combine(carry, excl, frame_len);
     carry = combine(carry, total, frame_len);
-    int32_t t[kFrItems], h[kFrItems], w[kFrItems];
+    const bool inside = g >= lo && g + kFrItems <= hi;
+    if (mine.n == 0 && (pre.n == 0 || p_base - pre.last > rows + 2)) {
+      // no marker among the thread's tokens and none of them inside a frame:
+      // all text, (p + off) on every plane
+      const int32_t off =
+          pre.n == 0 ? 0
+                     : pre.first + (pre.n - 1) * span32 + pre.gaps + span32 - frame_len - pre.last;
+      const int32_t b = p_base + off;
+      if (inside) {
 #pragma unroll
-    for (int j = 0; j < kFrItems; ++j) {
-      const int32_t p = static_cast<int32_t>(g + j - sl.first);  // local index
-      if (v[j] == marker) pre = combine(pre, Summary{1, p, p, 0}, frame_len);
-      int32_t pt, ph, pw;
-      if (pre.n == 0) {
-        pt = ph = pw = p;
-      } else {
-        const int32_t anchor = pre.first + (pre.n - 1) * span32 + pre.gaps;
-        const int32_t d = p - pre.last;  // offset into the last frame opened
-        if (d == 0) {
-          pt = anchor;
-          ph = pw = anchor - 1;
-        } else if (d <= rows) {
-          const uint32_t k = static_cast<uint32_t>(d - 1);
-          const uint32_t q = k / uside;
-          pt = anchor;
-          ph = anchor + static_cast<int32_t>(q);
-          pw = anchor + static_cast<int32_t>(k - q * uside);
-        } else if (d == rows + 1) {
-          pt = anchor;
-          ph = pw = anchor + side;
-        } else if (d == rows + 2) {
-          pt = ph = pw = anchor;
-        } else {
-          pt = ph = pw = anchor + span32 + (d - frame_len);
+        for (int r = 0; r < 3; ++r) {
+          store4(pos + r * n_tokens + g, b, b + 1, b + 2, b + 3);
+          store4(pos + r * n_tokens + g + 4, b + 4, b + 5, b + 6, b + 7);
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kFrItems; ++j)
+          if (g + j >= lo && g + j < hi)
+            for (int r = 0; r < 3; ++r) __stcs(pos + r * n_tokens + g + j, b + j);
       }
-      t[j] = pt;
-      h[j] = ph;
-      w[j] = pw;
+      continue;
     }
-    int32_t* const planes[3] = {pos + g, pos + n_tokens + g, pos + 2 * n_tokens + g};
-    const int32_t* const vals[3] = {t, h, w};
-    if (vec && g >= lo && g + kFrItems <= hi) {
+    // the planes of the thread's tokens, four at a time
 #pragma unroll
-      for (int r = 0; r < 3; ++r) {
-        int4* dst = reinterpret_cast<int4*>(planes[r]);
-        dst[0] = make_int4(vals[r][0], vals[r][1], vals[r][2], vals[r][3]);
-        dst[1] = make_int4(vals[r][4], vals[r][5], vals[r][6], vals[r][7]);
+    for (int half = 0; half < kFrItems / 4; ++half) {
+      int32_t t[4], h[4], w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int j = 4 * half + i;
+        const int32_t p = p_base + j;  // local index
+        if (v[j] == marker) pre = combine(pre, Summary{1, p, p, 0}, frame_len);
+        int32_t pt, ph, pw;
+        if (pre.n == 0) {
+          pt = ph = pw = p;
+        } else {
+          const int32_t anchor = pre.first + (pre.n - 1) * span32 + pre.gaps;
+          const int32_t d = p - pre.last;  // offset into the last frame opened
+          if (d == 0) {
+            pt = anchor;
+            ph = pw = anchor - 1;
+          } else if (d <= rows) {
+            // row k = d - 1 of the grid: k / side by a multiply-high with
+            // ceil(2^32 / side), exact since k * side < side^3 <= 2^21
+            const uint32_t k = static_cast<uint32_t>(d - 1);
+            const uint32_t q = __umulhi(k, side_magic);
+            pt = anchor;
+            ph = anchor + static_cast<int32_t>(q);
+            pw = anchor + static_cast<int32_t>(k - q * static_cast<uint32_t>(side));
+          } else if (d == rows + 1) {
+            pt = anchor;
+            ph = pw = anchor + side;
+          } else if (d == rows + 2) {
+            pt = ph = pw = anchor;
+          } else {
+            pt = ph = pw = anchor + span32 + (d - frame_len);
+          }
+        }
+        t[i] = pt;
+        h[i] = ph;
+        w[i] = pw;
       }
-    } else {
+      const int64_t gh = g + 4 * half;
+      int32_t* const planes[3] = {pos + gh, pos + n_tokens + gh, pos + 2 * n_tokens + gh};
+      const int32_t* const vals[3] = {t, h, w};
+      if (inside) {
 #pragma unroll
-      for (int j = 0; j < kFrItems; ++j)
-        if (g + j >= lo && g + j < hi)
-          for (int r = 0; r < 3; ++r) planes[r][j] = vals[r][j];
+        for (int r = 0; r < 3; ++r)
+          store4(planes[r], vals[r][0], vals[r][1], vals[r][2], vals[r][3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (gh + i >= lo && gh + i < hi)
+            for (int r = 0; r < 3; ++r) __stcs(planes[r] + i, vals[r][i]);
+      }
+    }
+  }
+  if (writer && threadIdx.x == 0) {
+    // an empty prompt ran no chunk: its carry is slice 0's, the identity
+    if (carry.n == 0) {
+      out_start[blockIdx.x] = kTextOnlyStart;
+      out_amount[blockIdx.x] = 0;
+    } else {
+      const int64_t span = side + 1;
+      const int64_t start = static_cast<int64_t>(carry.last) + frame_len;
+      const int64_t anchor = carry.first + static_cast<int64_t>(carry.n - 1) * span + carry.gaps;
+      out_start[blockIdx.x] = static_cast<int32_t>(start);
+      out_amount[blockIdx.x] = static_cast<int32_t>(start - (anchor + span));
     }
   }
 }
@@ -379,13 +498,19 @@ cudaError_t launch_positions_frames(const int32_t* ids, const int32_t* cu_seqlen
   const dim3 grid(static_cast<unsigned>(num_seqs), static_cast<unsigned>(slices));
   Summary* work = static_cast<Summary*>(workspace);
   const int32_t frame_len = grid_side * grid_side + 3;
-  frames_summary_kernel<<<grid, kFrThreads, 0, stream>>>(ids, cu_seqlens, num_seqs, n_tokens,
-                                                         image_token_id, frame_len, work,
-                                                         device_status);
+  const dim3 sum_grid(static_cast<unsigned>(num_seqs),
+                      static_cast<unsigned>((slices + kFrSumSlices - 1) / kFrSumSlices));
+  frames_summary_kernel<<<sum_grid, kFrThreads, 0, stream>>>(
+      ids, cu_seqlens, num_seqs, n_tokens, image_token_id, frame_len,
+      static_cast<int32_t>(slices), work, device_status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // ceil(2^32 / side); side 1 has only grid row 0, for which 0 serves
+  const uint32_t side_magic =
+      grid_side == 1 ? 0u
+                     : static_cast<uint32_t>(((uint64_t{1} << 32) + grid_side - 1) / grid_side);
   return pdl::launch(frames_positions_kernel, grid, dim3(kFrThreads), 0, stream, true, ids,
-                     cu_seqlens, num_seqs, n_tokens, image_token_id, grid_side,
+                     cu_seqlens, num_seqs, n_tokens, image_token_id, grid_side, side_magic,
                      static_cast<const Summary*>(work), out_pos, out_start, out_amount);
 }
 

@@ -101,10 +101,21 @@ __global__ void __launch_bounds__(kThreads, BatchShape<kBatch>::kMinBlocksPerSm)
   // Planes of the current item's token, loaded one item ahead so that their
   // latency overlaps the previous item's head rows.
   int32_t p0 = 0, p1 = 0, p2 = 0;
+  // The first token's sequence and index come from cu_seqlens (and
+  // pos_offset), which the kernels this one may be launched behind never
+  // write: that search runs before the wait below.
+  int32_t seq = 0;
+  int64_t idx = 0;
+  if (kFromShift && v < n_items) token_seq(args, G == 1 ? v : v % N, seq, idx);
   // Launched programmatically behind the positions kernels, pos (or the
   // shift state) is only ready after this wait; otherwise it returns at once.
   pdl::wait();
-  if (v < n_items) token_planes<kFromShift>(args, G == 1 ? v : v % N, p0, p1, p2);
+  if (v < n_items) {
+    if constexpr (kFromShift)
+      shift_planes(args, seq, idx, p0, p1, p2);
+    else
+      token_planes<false>(args, G == 1 ? v : v % N, p0, p1, p2);
+  }
   for (; v < n_items; v += v_step) {
     const int64_t g = (G == 1) ? 0 : v / N;
     const int64_t t = v - g * N;

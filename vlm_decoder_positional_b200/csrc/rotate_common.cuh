@@ -83,6 +83,17 @@ __device__ __forceinline__ void store_planes(const RotateArgs& a, int64_t t, int
   a.pos_out[2 * a.n_tokens + t] = p2;
 }
 
+// Planes of the token at absolute index p of sequence b, from the sequence's
+// shift state.  start / amount may come from the kernel just before (the
+// one-call path's origin scan): read through L2, not the read-only path.
+__device__ __forceinline__ void shift_planes(const RotateArgs& a, int32_t b, int64_t p,
+                                             int32_t& p0, int32_t& p1, int32_t& p2) {
+  const Planes r = canvas_row(p, __ldcg(a.start + b), __ldcg(a.amount + b));
+  p0 = r.t;
+  p1 = r.h;
+  p2 = r.w;
+}
+
 template <bool kFromShift>
 __device__ __forceinline__ void token_planes(const RotateArgs& a, int64_t t, int32_t& p0,
                                              int32_t& p1, int32_t& p2) {
@@ -94,12 +105,7 @@ __device__ __forceinline__ void token_planes(const RotateArgs& a, int64_t t, int
     int32_t b;
     int64_t p;
     token_seq(a, t, b, p);
-    // start / amount may come from the kernel just before (the one-call
-    // path's origin scan): read through L2, not the read-only path
-    const Planes r = canvas_row(p, __ldcg(a.start + b), __ldcg(a.amount + b));
-    p0 = r.t;
-    p1 = r.h;
-    p2 = r.w;
+    shift_planes(a, b, p, p0, p1, p2);
   }
 }
 

@@ -144,14 +144,24 @@ __global__ void __launch_bounds__(kThreads)
   const int tl = (threadIdx.x >> 5) * 8 + ((lane >> 3) | (((lane >> 2) & 1) << 2));
   const int64_t t = static_cast<int64_t>(t0) + tl;
   int32_t p0 = 0, p1 = 0, p2 = 0;  // rows past the last token are zeros and are not stored
+  // The token's sequence and index come from cu_seqlens (and pos_offset),
+  // which the kernels this one may be launched behind never write: the
+  // search's chain of dependent loads runs before the wait below.
+  int32_t seq = 0;
+  int64_t idx = 0;
+  if (kFromShift && t < args.r.n_tokens) token_seq(args.r, t, seq, idx);
   // Launched programmatically behind the positions kernels, the producer's
   // loads of Q and K (which those kernels never touch) are already under way;
   // pos (or the shift state) is ready after this wait.  Otherwise it returns
   // at once.
   pdl::wait();
   if (t < args.r.n_tokens) {
-    token_planes<kFromShift>(args.r, t, p0, p1, p2);
-    if (kFromShift && args.r.pos_out != nullptr && u == 0) store_planes(args.r, t, p0, p1, p2);
+    if constexpr (kFromShift) {
+      shift_planes(args.r, seq, idx, p0, p1, p2);
+      if (args.r.pos_out != nullptr && u == 0) store_planes(args.r, t, p0, p1, p2);
+    } else {
+      token_planes<false>(args.r, t, p0, p1, p2);
+    }
   }
   float c[8], s[8];
 #pragma unroll
