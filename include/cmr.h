@@ -170,7 +170,7 @@ CMR_API cmr_status cmr_positions_chunk(const int32_t* ids, const int32_t* cu_seq
  *   workspace      device memory, 16-byte aligned, of workspace_bytes >= 16 *
  *                  num_seqs; cmr_positions_frames_workspace_bytes gives the
  *                  size for full parallelism (16 B per sequence per slice of
- *                  about 2,048 tokens); a smaller one works with fewer,
+ *                  about 4,096 tokens); a smaller one works with fewer,
  *                  longer slices.  It holds one summary per slice between the
  *                  call's two kernels; its contents before and after a call
  *                  do not matter, but calls that overlap on the device must

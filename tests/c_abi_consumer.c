@@ -52,7 +52,7 @@ static int host_checks(void) {
   CHECK(cmr_positions_rotate_qk(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL, 1, 8, 2,
                                 256, 1e7, bad_sections, 64, NULL, NULL) == CMR_EINVAL);
   /* several frames per prompt: the workspace size and the host checks */
-  CHECK(cmr_positions_frames_workspace_bytes(32, 32 * 8192) == 16u * 32 * 4);
+  CHECK(cmr_positions_frames_workspace_bytes(32, 32 * 8192) == 16u * 32 * 2);
   CHECK(cmr_positions_frames(fake, fake, 1, 10, 248078, 0, fake, fake, fake, fake, 1 << 20, NULL,
                              NULL) == CMR_EINVAL);
   CHECK(cmr_positions_frames_noalloc(fake, fake, 16385, 16385, 248078, 8, fake, fake, fake, NULL,

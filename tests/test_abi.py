@@ -138,11 +138,11 @@ def test_positions_frames_rejects_bad_arguments_on_the_host(lib, kw):
 
 
 def test_positions_frames_workspace_size():
-    # 16 bytes per sequence per slice of about 2,048 tokens
+    # 16 bytes per sequence per slice of about 4,096 tokens
     assert cmr.positions_frames_workspace_bytes(0, 0) == 0
     assert cmr.positions_frames_workspace_bytes(1, 80) == 16
-    assert cmr.positions_frames_workspace_bytes(32, 32 * 8192) == 16 * 32 * 4
-    assert cmr.positions_frames_workspace_bytes(1, 300_000) == 16 * 147
+    assert cmr.positions_frames_workspace_bytes(32, 32 * 8192) == 16 * 32 * 2
+    assert cmr.positions_frames_workspace_bytes(1, 300_000) == 16 * 74
     assert lib_ok(cmr.lib().cmr_positions_frames(None, None, 0, 0, 248078, 8, None, None, None,
                                                  None, 0, None, None))
 

@@ -56,7 +56,7 @@ def test_no_alloc_entry_point_matches_the_workspace_one_in_a_row(cuda_device):
     # each), shorter ones at s = 16 (one slice each), and 9,000 prompts whose
     # two slices each would not fit the scratch (one slice each instead)
     for seed, s, n_prompts, max_len in ((1, 8, 24, 30000), (2, 16, 300, 3000),
-                                        (3, 8, 9000, 4200)):
+                                        (3, 8, 9000, 9000)):
         ids_np, cu_np = batch(seed, s, n_prompts, max_len)
         ids, cu = t32(ids_np, dev), t32(cu_np, dev)
         got = no_alloc_call(ids, cu, s, dev)

@@ -17,20 +17,18 @@
 // so token p needs only the inclusive prefix, over the tokens up to p, of
 // (marker count, first marker, last marker, summed excess gaps) -- an
 // associative (not commutative) combine.  Each prompt b is cut into slices
-// of about 2,048 tokens, and two kernels run over them:
-//   1. frames_summary_kernel, CTAs (b, group of kFrSumSlices slices), reduces
-//      each slice's tokens to that 16-byte summary in a caller-provided
-//      workspace [num_seqs][slices]; the first ids of all its slices are in
-//      flight before it folds any;
-//   2. frames_positions_kernel, CTAs (b, slice), launched programmatically
-//      behind it, loads its first ids before it waits for the summaries, has
-//      one warp fold the summaries of the slices before its own into a carry,
-//      then walks its slice in chunks of kFrThreads x kFrItems tokens: each
-//      thread folds its own kFrItems consecutive tokens, one block scan of
-//      the threads' summaries gives each thread its prefix, and the thread
-//      walks its tokens again writing their planes.  The CTA holding the
-//      prompt's last token ends with the whole prompt's summary and writes
-//      its state.
+// of about 4,096 tokens, and two kernels run over CTAs (b, slice):
+//   1. frames_summary_kernel reduces its slice's tokens to that 16-byte
+//      summary in a caller-provided workspace [num_seqs][slices], with the
+//      ids of kFrSumUnroll block steps in flight before it folds any;
+//   2. frames_positions_kernel, launched programmatically behind it, loads its
+//      first ids before it waits for the summaries, has one warp fold the
+//      summaries of the slices before its own into a carry, then walks its
+//      slice in chunks of kFrThreads x kFrItems tokens: each thread folds its
+//      own kFrItems consecutive tokens, one block scan of the threads'
+//      summaries gives each thread its prefix, and the thread walks its
+//      tokens again writing their planes.  The CTA holding the prompt's last
+//      token ends with the whole prompt's summary and writes its state.
 // Each thread owns 8 consecutive tokens at an 8-aligned index of the packed
 // batch, so ids are read as 16-byte vectors and each plane row is written in
 // the widest stores its alignment allows (16 bytes when n_tokens is a
@@ -52,9 +50,9 @@ constexpr int kFrThreads = 256;
 constexpr int kFrWarps = kFrThreads / 32;
 constexpr int kFrItems = 8;                                  // consecutive tokens per thread
 constexpr int kFrChunk = kFrThreads * kFrItems;              // 2048 tokens per block step
-constexpr int kFrSliceTarget = kFrChunk;                     // tokens per CTA (target)
+constexpr int kFrSliceTarget = 2 * kFrChunk;                 // tokens per slice (target)
 constexpr int kFrMaxSlices = 65535;                          // gridDim.y limit
-constexpr int kFrSumSlices = 4;                              // slices per summary CTA
+constexpr int kFrSumUnroll = 2;                              // summary block steps in flight
 constexpr int kFrPosBlocks = 5;                              // positions CTAs per SM
 
 // Prefix summary of a run of tokens: n markers, the first and last of them
@@ -204,21 +202,27 @@ __device__ __forceinline__ void fr_range(uint32_t y, uint32_t slices, FrSlice* s
   sl->p1 = static_cast<int32_t>(min(len, static_cast<uint32_t>(sl->p0) + per));
 }
 
-// The summary of the marker tokens among v (local indices from p_base).
+// The summary of the marker tokens among v (local indices from p_base): a
+// bit mask of the markers first, so that a group without one (nearly all of
+// them) costs a compare per token.
 __device__ __forceinline__ Summary fold_group(const int32_t (&v)[kFrItems], int32_t p_base,
                                               int32_t marker, int32_t frame_len) {
-  Summary mine{0, 0, 0, 0};
+  uint32_t m = 0;
 #pragma unroll
-  for (int j = 0; j < kFrItems; ++j)
-    if (v[j] == marker) mine = combine(mine, Summary{1, p_base + j, p_base + j, 0}, frame_len);
+  for (int j = 0; j < kFrItems; ++j) m |= static_cast<uint32_t>(v[j] == marker) << j;
+  Summary mine{0, 0, 0, 0};
+  while (m != 0) {
+    const int32_t p = p_base + __ffs(m) - 1;
+    m &= m - 1;
+    mine = combine(mine, Summary{1, p, p, 0}, frame_len);
+  }
   return mine;
 }
 
 __global__ void __launch_bounds__(kFrThreads)
     frames_summary_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                           int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t frame_len,
-                          int32_t slices, Summary* __restrict__ work,
-                          int32_t* __restrict__ status) {
+                          Summary* __restrict__ work, int32_t* __restrict__ status) {
   __shared__ BlockBufs bufs;
   int turn = 0;
   pdl::launch_dependents();
@@ -229,36 +233,28 @@ __global__ void __launch_bounds__(kFrThreads)
       atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
     return;
   }
-  // this CTA's slices y0 .. y0 + kFrSumSlices - 1, each walked in 8-aligned
-  // groups of kFrItems tokens (global indices of the packed batch), kFrChunk
-  // tokens per block step; the first group of every slice is loaded before
-  // any is folded
-  const uint32_t y0 = blockIdx.y * kFrSumSlices;
-  int32_t v[kFrSumSlices][kFrItems];
-  int64_t lo[kFrSumSlices], hi[kFrSumSlices];
+  // the slice as global indices of the packed batch, walked in 8-aligned
+  // groups of kFrItems tokens, kFrChunk tokens per block step; the groups of
+  // kFrSumUnroll steps are loaded before any is folded
+  fr_range(blockIdx.y, gridDim.y, &sl);
+  const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
+  Summary run{0, 0, 0, 0};
+  for (int64_t c = lo & ~static_cast<int64_t>(kFrItems - 1); c < hi;
+       c += kFrSumUnroll * kFrChunk) {
+    int32_t v[kFrSumUnroll][kFrItems];
 #pragma unroll
-  for (int r = 0; r < kFrSumSlices; ++r) {
-    fr_range(y0 + r, static_cast<uint32_t>(slices), &sl);
-    lo[r] = sl.first + sl.p0;
-    hi[r] = y0 + r < static_cast<uint32_t>(slices) ? sl.first + sl.p1 : lo[r];
-    const int64_t c = lo[r] & ~static_cast<int64_t>(kFrItems - 1);
-    load_group<false>(ids, c + static_cast<int64_t>(threadIdx.x) * kFrItems, lo[r], hi[r],
-                      ~marker, v[r]);
-  }
+    for (int u = 0; u < kFrSumUnroll; ++u)
+      load_group<false>(ids, c + u * kFrChunk + static_cast<int64_t>(threadIdx.x) * kFrItems, lo,
+                        hi, ~marker, v[u]);
 #pragma unroll
-  for (int r = 0; r < kFrSumSlices; ++r) {
-    if (y0 + r >= static_cast<uint32_t>(slices)) break;  // the same for every thread
-    Summary run{0, 0, 0, 0};
-    for (int64_t c = lo[r] & ~static_cast<int64_t>(kFrItems - 1); c < hi[r]; c += kFrChunk) {
-      const int64_t g = c + static_cast<int64_t>(threadIdx.x) * kFrItems;
-      if (c != (lo[r] & ~static_cast<int64_t>(kFrItems - 1)))
-        load_group<false>(ids, g, lo[r], hi[r], ~marker, v[r]);
-      const Summary mine =
-          fold_group(v[r], static_cast<int32_t>(g - sl.first), marker, frame_len);
+    for (int u = 0; u < kFrSumUnroll; ++u) {
+      if (c + u * kFrChunk >= hi) break;  // the same for every thread
+      const int64_t g = c + u * kFrChunk + static_cast<int64_t>(threadIdx.x) * kFrItems;
+      const Summary mine = fold_group(v[u], static_cast<int32_t>(g - sl.first), marker, frame_len);
       run = combine(run, block_reduce(mine, frame_len, bufs, turn), frame_len);
     }
-    if (threadIdx.x == 0) work[static_cast<int64_t>(blockIdx.x) * slices + y0 + r] = run;
   }
+  if (threadIdx.x == 0) work[static_cast<int64_t>(blockIdx.x) * gridDim.y + blockIdx.y] = run;
 }
 
 // Ordered fold of summaries[0, count) by one warp (all 32 lanes call it);
@@ -498,11 +494,9 @@ cudaError_t launch_positions_frames(const int32_t* ids, const int32_t* cu_seqlen
   const dim3 grid(static_cast<unsigned>(num_seqs), static_cast<unsigned>(slices));
   Summary* work = static_cast<Summary*>(workspace);
   const int32_t frame_len = grid_side * grid_side + 3;
-  const dim3 sum_grid(static_cast<unsigned>(num_seqs),
-                      static_cast<unsigned>((slices + kFrSumSlices - 1) / kFrSumSlices));
-  frames_summary_kernel<<<sum_grid, kFrThreads, 0, stream>>>(
-      ids, cu_seqlens, num_seqs, n_tokens, image_token_id, frame_len,
-      static_cast<int32_t>(slices), work, device_status);
+  frames_summary_kernel<<<grid, kFrThreads, 0, stream>>>(ids, cu_seqlens, num_seqs, n_tokens,
+                                                         image_token_id, frame_len, work,
+                                                         device_status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // ceil(2^32 / side); side 1 has only grid row 0, for which 0 serves
