@@ -523,9 +523,11 @@ def run_ours(args):
         e2e = {"skipped": f"--op {args.op} times the device step only; the end-to-end path "
                           "is measured with --op rotate"}
 
-    ceiling = None
+    ceiling = same_size_copy = None
     if args.op == "rotate" and kernel_ran == "rotate_qk_staged_kernel":
         ceiling = run_copy_pattern_probe(wl, dev, stream)
+    if args.op == "rotate":
+        same_size_copy = run_plain_copy_probe(rot_b, dev, stream)
 
     if rank == 0:
         peak, peak_src = measured_peak()
@@ -554,6 +556,10 @@ def run_ours(args):
             roofline["ceiling"] = ceiling["gbs"]
             roofline["frac_of_ceiling"] = achieved / ceiling["gbs"]
             roofline["ceiling_source"] = ceiling["what"]
+        if same_size_copy is not None:
+            roofline["same_size_copy"] = same_size_copy["gbs"]
+            roofline["frac_of_same_size_copy"] = achieved / same_size_copy["gbs"]
+            roofline["same_size_copy_source"] = same_size_copy["what"]
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -621,18 +627,50 @@ def run_copy_pattern_probe(wl, dev, stream, launches=10, warmup=3):
                     "loaded and stored back unchanged, no math; mean of %d launches" % launches}
 
 
+def run_plain_copy_probe(moved, dev, stream, launches=10, warmup=3):
+    """A plain device-to-device copy (torch copy_, read + write bytes) of the
+    same total bytes as the rotation moves, timed the same way: the copy peak
+    at this launch size, which includes the start and drain one launch of
+    this size cannot hide."""
+    half = (moved // 2 + 15) // 16 * 16
+    src = torch.empty(half, dtype=torch.uint8, device=dev)
+    dst = torch.empty(half, dtype=torch.uint8, device=dev)
+    src.fill_(1)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            dst.copy_(src)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(launches)]
+        torch.cuda.synchronize(dev)
+        for a, z in ev:
+            a.record(stream)
+            dst.copy_(src)
+            z.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(z) for a, z in ev)
+    del src, dst
+    return {"gbs": 2 * half / (ms / 1e3) / 1e9, "ms": ms, "bytes": 2 * half,
+            "what": "torch copy_ of the same read + write bytes as one launch moves (two "
+                    "contiguous buffers); mean of %d copies" % launches}
+
+
 def run_probe_only(args):
     """--probe copy-pattern: the ceiling probe alone on the workload's Q/K."""
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     wl = inputs.make_config(args.workload, device=dev)
-    res = run_copy_pattern_probe(wl, dev, torch.cuda.current_stream(dev), launches=args.steps,
+    stream = torch.cuda.current_stream(dev)
+    res = run_copy_pattern_probe(wl, dev, stream, launches=args.steps, warmup=args.warmup)
+    plain = run_plain_copy_probe(res["bytes"], dev, stream, launches=args.steps,
                                  warmup=args.warmup)
     peak, src = measured_peak()
     print(json.dumps({"probe": "copy-pattern", "workload": workload_label(wl),
                       "gbs": res["gbs"], "ms_per_launch": res["ms"], "bytes": res["bytes"],
                       "peak": peak, "peak_source": src, "frac_of_peak": res["gbs"] / peak,
-                      "launches": args.steps, "what": res["what"]}), flush=True)
+                      "launches": args.steps, "what": res["what"],
+                      "same_size_copy_gbs": plain["gbs"],
+                      "same_size_copy_frac_of_peak": plain["gbs"] / peak,
+                      "same_size_copy_what": plain["what"]}), flush=True)
     return 0
 
 
