@@ -94,6 +94,70 @@ def test_long_single_prompt_spans_many_ctas(cuda_device):
         check_batch(ids, np.array([0, 300_000], np.int32), cuda_device)
 
 
+BLOCK = 16_384  # ids per block of the origin scan
+
+
+@pytest.mark.parametrize("length", [120_000, 200_000, 300_000, 1_000_000])
+def test_cluster_scan_block_and_rank_boundaries(cuda_device, length):
+    # prompts this long average more than four blocks of ids, so each one is
+    # scanned by a cluster of 2, 4 or 8 CTAs dealing the blocks round-robin;
+    # markers sit on both sides of every block edge the prompt has (so on
+    # every rank and round), first and last, or nowhere
+    rng = np.random.default_rng(10 + length // 1000)
+    blocks = (length + BLOCK - 1) // BLOCK
+    origins = {-1, 0, 1, length - 1, length - 67, length // 2}
+    for j in range(1, blocks):
+        origins.update({j * BLOCK - 1, j * BLOCK, j * BLOCK + BLOCK // 2})
+    origins = sorted(o for o in origins if -1 <= o < length)
+    if length >= 300_000:  # a sample of the edges keeps the batch small
+        origins = origins[:: 3 if length < 1_000_000 else 5] + [-1]
+    prompts = [inputs.prompt_ids(rng, length, o) for o in origins]
+    # a later marker does not hide an earlier one: extra markers after O
+    for p, o in zip(prompts, origins):
+        if 0 <= o < length - 100:
+            p[rng.integers(o + 68, length, size=5)] = MARK
+    ids, cu = inputs.pack(prompts)
+    check_batch(ids, cu, cuda_device)
+
+
+def test_cluster_scan_with_short_and_empty_prompts_in_the_batch(cuda_device):
+    # a long average (clusters of 8) with short and empty prompts among the
+    # long ones: the ranks past a short prompt's end scan nothing
+    rng = np.random.default_rng(20)
+    lens = [300_000, 0, 5, 70, 300_000, 1, 200_000, 0]
+    origins = [200_000, -1, 2, 0, -1, 0, 16_384 * 7 + 3, -1]
+    prompts = [inputs.prompt_ids(rng, n, o) for n, o in zip(lens, origins)]
+    ids, cu = inputs.pack(prompts)
+    check_batch(ids, cu, cuda_device)
+
+
+def test_cluster_scan_in_chunks_and_the_one_call_path(cuda_device):
+    # the continuation form over long chunks (clusters), with sequences whose
+    # frame is already known (no scan) beside ones still text-only, and the
+    # one-call path's origin scan on long prompts
+    dev = cuda_device
+    rng = np.random.default_rng(30)
+    n = 150_000
+    prompts = [inputs.prompt_ids(rng, n, o) for o in (-1, 70_000, -1, 131_072)]
+    ids_np, cu_np = inputs.pack(prompts)
+    offset = np.array([0, 1000, 5000, 0], np.int32)
+    in_start = np.array([1 << 30, 1 << 30, 4000, 1 << 30], np.int32)
+    in_amount = np.array([0, 0, 3942, 0], np.int32)
+    want = oracle.positions_chunk(ids_np, cu_np, MARK, pos_offset=offset, in_start=in_start,
+                                  in_amount=in_amount)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+    got = cmr.positions_chunk(t(ids_np), t(cu_np), pos_offset=t(offset),
+                              state=(t(in_start), t(in_amount)))
+    for g, w in zip(got, want):
+        np.testing.assert_array_equal(g.cpu().numpy(), w)
+    q = inputs.random_qk((1, ids_np.shape[0], 2, 256), 31, dev)
+    k = inputs.random_qk((1, ids_np.shape[0], 1, 256), 32, dev)
+    pos, start, amount = cmr.positions_rotate_qk(t(ids_np), t(cu_np), q, k)
+    want = oracle.positions(ids_np, cu_np, MARK)
+    for g, w in zip((pos, start, amount), want):
+        np.testing.assert_array_equal(g.cpu().numpy(), w)
+
+
 def test_many_short_prompts_and_repeated_markers(cuda_device):
     rng = np.random.default_rng(4)
     lens = rng.integers(0, 90, size=5000)

@@ -8,12 +8,14 @@
 // the LiteRT card's runtime uses plain 1-D positions; both are selectable.
 //
 // Work split: two kernels.
-//   1. canvas_origin_kernel, one CTA per prompt chunk, finds the chunk's first
-//      marker (16 loads in flight per thread, warp `redux.sync` min, a
-//      shared-memory min) and stops at the first block of ids that holds one,
-//      so no id is read twice; it writes the chunk's outgoing state (start,
-//      amount) -- carried over when a frame is already known, (2^30, 0) for
-//      text and for the 1-D rule.
+//   1. canvas_origin_kernel, one CTA per prompt chunk (or, for long chunks, a
+//      cluster of K CTAs that deal the blocks of ids round-robin and exchange
+//      their minima through distributed shared memory after each round),
+//      finds the chunk's first marker (16 loads in flight per thread, warp
+//      `redux.sync` min, a shared-memory min) and stops at the first block
+//      (round) of ids that holds one, so no id is read twice; it writes the
+//      chunk's outgoing state (start, amount) -- carried over when a frame is
+//      already known, (2^30, 0) for text and for the 1-D rule.
 //   2. canvas_positions_kernel, CTAs (b, s) over slices of about 2,048 tokens,
 //      launched programmatically behind the first (it starts while the scan
 //      runs and waits for it before reading the state), writes the planes:
@@ -22,10 +24,14 @@
 // through the caller's out_start / out_amount.  The one-call path
 // (cmr_positions_rotate_qk) launches only the first kernel and lets the
 // rotation write the planes.
+#include <cooperative_groups.h>
+
 #include <climits>
 
 #include "canvas.cuh"
 #include "pdl.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace cmr {
 namespace {
@@ -37,34 +43,101 @@ constexpr int kPosThreads = 512;
 constexpr int kSliceTarget = 2048;                          // tokens per planes CTA
 constexpr int kMaxSlices = 65535;                           // gridDim.y limit
 constexpr int kQwenVlFrameShift = kGridRows + 1;            // start = O + 65
+constexpr int kOriginMaxCluster = 8;                        // CTAs per long chunk
+
+// The ids of the block seq[c, c + kScanChunk) this thread reads (16 loads in
+// flight), entries past len reading as a non-marker.
+__device__ __forceinline__ void load_block(const int32_t* __restrict__ seq, int64_t c,
+                                           int64_t len, int32_t marker,
+                                           int32_t (&v)[kIdsPerThread]) {
+#pragma unroll
+  for (int m = 0; m < kIdsPerThread; ++m) {
+    const int64_t e = c + m * kOriginThreads + threadIdx.x;
+    v[m] = (e < len) ? __ldg(seq + e) : ~marker;
+  }
+}
+
+// Smallest offset in a block of ids (loaded by load_block) whose id is the
+// marker, or INT_MAX.  Block-uniform result; all threads of the CTA must call
+// it.
+__device__ __forceinline__ int block_min(const int32_t (&v)[kIdsPerThread], int32_t marker,
+                                         int* s_warp_min) {
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int best = INT_MAX;  // offset within the block; smaller m = smaller index
+#pragma unroll
+  for (int m = kIdsPerThread - 1; m >= 0; --m)
+    if (v[m] == marker) best = m * kOriginThreads + threadIdx.x;
+  best = __reduce_min_sync(0xffffffffu, best);
+  if (lane == 0) s_warp_min[warp] = best;
+  __syncthreads();
+  int block_best = INT_MAX;
+#pragma unroll
+  for (int i = 0; i < kOriginThreads / 32; ++i) block_best = min(block_best, s_warp_min[i]);
+  __syncthreads();  // s_warp_min is rewritten by the next block
+  return block_best;
+}
 
 // Smallest local index in seq[0, len) whose id is the marker, or -1.
 // Block-uniform result; all threads of the CTA must call it.
 __device__ __forceinline__ int64_t first_marker(const int32_t* __restrict__ seq, int64_t len,
                                                 int32_t marker, int* s_warp_min) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
   for (int64_t c = 0; c < len; c += kScanChunk) {
     int32_t v[kIdsPerThread];
-#pragma unroll
-    for (int m = 0; m < kIdsPerThread; ++m) {
-      const int64_t e = c + m * kOriginThreads + threadIdx.x;
-      v[m] = (e < len) ? __ldg(seq + e) : ~marker;
-    }
-    int best = INT_MAX;  // offset within the chunk; smaller m = smaller index
-#pragma unroll
-    for (int m = kIdsPerThread - 1; m >= 0; --m)
-      if (v[m] == marker) best = m * kOriginThreads + threadIdx.x;
-    best = __reduce_min_sync(0xffffffffu, best);
-    if (lane == 0) s_warp_min[warp] = best;
-    __syncthreads();
-    int block_best = INT_MAX;
-#pragma unroll
-    for (int i = 0; i < kOriginThreads / 32; ++i) block_best = min(block_best, s_warp_min[i]);
-    __syncthreads();  // s_warp_min is rewritten by the next chunk
-    if (block_best != INT_MAX) return c + block_best;
+    load_block(seq, c, len, marker, v);
+    const int best = block_min(v, marker, s_warp_min);
+    if (best != INT_MAX) return c + best;
   }
   return -1;
+}
+
+// first_marker by the K CTAs of this CTA's cluster: in round i, rank r scans
+// block i * K + r; after each round lane q < K of warp 0 reads rank q's
+// minimum through distributed shared memory (double-buffered, so one cluster
+// barrier per round suffices), and the CTA's threads read the cluster's
+// minimum from warp 0; all stop at the first round that found a marker.
+// Each rank's loads for the next round are issued before that exchange, so
+// their latency overlaps it; no id is read twice, and at most one round past
+// the first marker is read.  Cluster-uniform result; every thread of every
+// CTA of the cluster must call it.  Local indices fit in int32 (a chunk's
+// length comes from int32 cu_seqlens).
+__device__ __forceinline__ int64_t first_marker_cluster(const int32_t* __restrict__ seq,
+                                                        int64_t len, int32_t marker,
+                                                        int* s_warp_min, int* s_found,
+                                                        int* s_all) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int64_t K = cluster.num_blocks();
+  const int64_t r = cluster.block_rank();
+  const int64_t blocks = (len + kScanChunk - 1) / kScanChunk;
+  int64_t result = -1;
+  int32_t v[kIdsPerThread];
+  load_block(seq, r * kScanChunk, len, marker, v);
+  for (int64_t i = 0; i * K < blocks; ++i) {
+    const int64_t c = (i * K + r) * kScanChunk;
+    int mine = INT_MAX;
+    if (c < len) {
+      const int best = block_min(v, marker, s_warp_min);
+      if (best != INT_MAX) mine = static_cast<int>(c + best);
+    }
+    if ((i + 1) * K < blocks) load_block(seq, c + K * kScanChunk, len, marker, v);
+    int* const slot = s_found + (i & 1);
+    if (threadIdx.x == 0) *slot = mine;
+    cluster.sync();
+    if (threadIdx.x < 32) {
+      const int q = threadIdx.x;
+      const int m = q < K ? *cluster.map_shared_rank(slot, q) : INT_MAX;
+      const int all = __reduce_min_sync(0xffffffffu, m);
+      if (q == 0) *s_all = all;
+    }
+    __syncthreads();
+    const int all = *s_all;  // rewritten only after the next round's block barriers
+    if (all != INT_MAX) {
+      result = all;
+      break;
+    }
+  }
+  cluster.sync();  // no CTA leaves while a peer may still read its s_found
+  return result;
 }
 
 // Bounds of prompt chunk b; false (uniform over the CTA) when cu_seqlens is
@@ -82,6 +155,9 @@ __device__ __forceinline__ bool chunk_bounds(const int32_t* __restrict__ cu, int
   return true;
 }
 
+// kCluster: launched in clusters of K CTAs per chunk (grid num_seqs * K);
+// otherwise one CTA per chunk.
+template <bool kCluster>
 __global__ void __launch_bounds__(kOriginThreads)
     canvas_origin_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ cu,
                          int32_t num_seqs, int64_t n_tokens, int32_t marker, int32_t rule,
@@ -90,11 +166,22 @@ __global__ void __launch_bounds__(kOriginThreads)
                          const int32_t* __restrict__ in_amount, int32_t* __restrict__ out_start,
                          int32_t* __restrict__ out_amount, int32_t* __restrict__ status) {
   __shared__ int s_warp_min[kOriginThreads / 32];
+  __shared__ int s_found[2];
+  __shared__ int s_all;
   pdl::launch_dependents();
-  const int32_t b = blockIdx.x;
+  // the chunk of this CTA (of its cluster), and whether it writes the results
+  int32_t b = blockIdx.x;
+  bool leader = true;
+  if constexpr (kCluster) {
+    cg::cluster_group cluster = cg::this_cluster();
+    b = static_cast<int32_t>(blockIdx.x / cluster.num_blocks());
+    leader = cluster.block_rank() == 0;
+  }
   int64_t first, len;
+  // every CTA of a cluster takes the same branches below (same chunk)
   if (!chunk_bounds(cu, num_seqs, n_tokens, b, &first, &len)) {
-    if (threadIdx.x == 0 && status != nullptr) atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
+    if (leader && threadIdx.x == 0 && status != nullptr)
+      atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
     return;
   }
   // The sequence's state before this chunk: (2^30, 0) while no frame is known.
@@ -104,7 +191,9 @@ __global__ void __launch_bounds__(kOriginThreads)
     start = kTextOnlyStart;
     amount = 0;
   } else if (start >= kTextOnlyStart) {
-    const int64_t m = first_marker(ids + first, len, marker, s_warp_min);
+    const int64_t m = kCluster ? first_marker_cluster(ids + first, len, marker, s_warp_min, s_found,
+                                                    &s_all)
+                               : first_marker(ids + first, len, marker, s_warp_min);
     if (m >= 0) {
       const int64_t origin = (pos_offset ? __ldg(pos_offset + b) : 0) + m;
       start = origin + (rule == CMR_RULE_QWEN_VL ? kQwenVlFrameShift : kFrameTokens);
@@ -114,7 +203,7 @@ __global__ void __launch_bounds__(kOriginThreads)
       amount = 0;
     }
   }
-  if (threadIdx.x == 0) {
+  if (leader && threadIdx.x == 0) {
     out_start[b] = static_cast<int32_t>(start);
     out_amount[b] = static_cast<int32_t>(amount);
   }
@@ -179,10 +268,31 @@ cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlen
                                    int32_t* out_start, int32_t* out_amount,
                                    int32_t* device_status, cudaStream_t stream) {
   if (num_seqs == 0) return cudaSuccess;
-  canvas_origin_kernel<<<static_cast<unsigned>(num_seqs), kOriginThreads, 0, stream>>>(
-      ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule, pos_offset, in_start, in_amount,
-      out_start, out_amount, device_status);
-  return cudaGetLastError();
+  // Chunks averaging more than four blocks of ids get a cluster of K CTAs
+  // (K a power of two up to kOriginMaxCluster, one per four blocks).
+  const int64_t avg = (n_tokens + num_seqs - 1) / num_seqs;
+  int k = 1;
+  while (k < kOriginMaxCluster && static_cast<int64_t>(k) * 4 * kScanChunk < avg) k *= 2;
+  if (k == 1) {
+    canvas_origin_kernel<false><<<static_cast<unsigned>(num_seqs), kOriginThreads, 0, stream>>>(
+        ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule, pos_offset, in_start,
+        in_amount, out_start, out_amount, device_status);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(static_cast<int64_t>(num_seqs) * k));
+  cfg.blockDim = dim3(kOriginThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(k);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, canvas_origin_kernel<true>, ids, cu_seqlens, num_seqs,
+                            n_tokens, image_token_id, rule, pos_offset, in_start, in_amount,
+                            out_start, out_amount, device_status);
 }
 
 cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
