@@ -227,6 +227,20 @@ def host_cores():
         return os.cpu_count() or 1
 
 
+def host_cpu():
+    """The host's CPU model (first /proc/cpuinfo entry) and logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count(), "threads_allowed": host_cores()}
+
+
 def oracle_sample_step(wl_cpu, n, threads=1):
     """One oracle pass over a sample: the planes of the prompts that hold the
     first n tokens (decode: of the first n prompts, then their new token),
@@ -302,7 +316,8 @@ def run_cpu_baseline(wl, seconds):
         out[threads] = (n / dt, sample_label(wl, n, threads) + f", {dt:.1f} s")
         del wl_cpu
     value, sample = out[cores]
-    res = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+    res = {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+           "host": host_cpu()}
     if cores > 1:
         res["single_thread"] = {"value": out[1][0], "sample": out[1][1]}
     return res
@@ -344,7 +359,8 @@ def run_reference(args):
                               cache_bytes(full_tokens, wl.num_layers, wl.hq, wl.hk, wl.rot_dim,
                                           wl.head_dim)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample + f", the fp64 oracle on {cores} host threads"},
+                         "sample": sample + f", the fp64 oracle on {cores} host threads",
+                         "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }), flush=True)
@@ -733,7 +749,7 @@ def run_frames_reference(args):
         "vs_baseline": None, "dtype": "int32", "data": "synthetic (seeded)",
         "config": frames_config(args, wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }), flush=True)
@@ -814,7 +830,7 @@ def run_frames(args):
                 take = min(b, take * 2)
                 t0 = time.perf_counter()
             cpu = {"value": int(wl.cu_seqlens[take]) / dt, "unit": UNIT, "cores": cores,
-                   "kind": "oracle",
+                   "kind": "oracle", "host": host_cpu(),
                    "sample": f"multi-frame planes of the first {take} prompts "
                              f"({int(wl.cu_seqlens[take])} tokens), 1 thread, {dt:.2f} s"}
         tokens_all = n * world
