@@ -302,6 +302,34 @@ CMR_API cmr_status cmr_positions_rotate_qk(const int32_t* ids, const int32_t* cu
                                            const int32_t sections[3], int32_t rot_dim,
                                            int32_t* device_status, cmr_stream_t stream);
 
+/* cmr_positions_rotate_qk on a batch that lives in host memory: the same
+ * arguments, results and errors, with ids, cu_seqlens, out_pos, out_start,
+ * out_amount, q and k all page-locked host memory mapped into the device's
+ * address space at the same address (cudaHostAlloc / cudaMallocHost, or
+ * cudaHostRegister with cudaHostRegisterMapped, on a system with unified
+ * addressing; PyTorch's pin_memory() tensors qualify).  The kernels read and
+ * write those buffers directly over PCIe (zero-copy): each id once, the
+ * rotated dims of each head row (rot_dim * 2 bytes of every head_dim * 2)
+ * read and written once, the planes and the state written once; the other
+ * dims of Q/K never cross the bus.  Nothing is staged in device memory and
+ * no copy engine is used, so a caller whose batch is on the host needs no
+ * device buffers and no copies of its own.  The rotation runs on the
+ * register kernel (plain loads and stores; tensor maps are never built over
+ * host memory).  Calls are asynchronous: the host may read the results, and
+ * must not touch the buffers, until the stream has been synchronised.
+ * device_status may be device memory or mapped host memory.
+ * Errors: as cmr_positions_rotate_qk, plus CMR_EINVAL for a buffer that is
+ * not mapped page-locked host memory (device memory and pageable host memory
+ * are refused). */
+CMR_API cmr_status cmr_positions_rotate_qk_host(const int32_t* ids, const int32_t* cu_seqlens,
+                                                int32_t num_seqs, int64_t n_tokens,
+                                                int32_t image_token_id, int32_t* out_pos,
+                                                int32_t* out_start, int32_t* out_amount, void* q,
+                                                void* k, int32_t num_layers, int32_t hq,
+                                                int32_t hk, int32_t head_dim, double theta,
+                                                const int32_t sections[3], int32_t rot_dim,
+                                                int32_t* device_status, cmr_stream_t stream);
+
 /* cmr_rotate_qk with the planes derived inside the kernel instead of read
  * from pos [3, n_tokens]: token t of prompt b (cu[b] <= t < cu[b+1]) sits at
  * absolute index p = pos_offset[b] + t - cu[b] and gets the canvas table's

@@ -28,7 +28,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     assert set(names) == {"cmr_positions", "cmr_positions_chunk", "cmr_positions_step",
-                          "cmr_rotate_qk", "cmr_positions_rotate_qk", "cmr_rotate_qk_shift",
+                          "cmr_rotate_qk", "cmr_positions_rotate_qk",
+                          "cmr_positions_rotate_qk_host", "cmr_rotate_qk_shift",
                           "cmr_rotate_qk_cache", "cmr_rotate_qk_kernel",
                           "cmr_rotate_qk_cache_kernel", "cmr_copy_rotated_dims",
                           "cmr_status_string", "cmr_last_error_message",
@@ -53,7 +54,7 @@ def test_status_strings_and_version(lib):
     for code in (0, 1, 2, 3):
         assert lib.cmr_status_string(code)
     assert b"unknown" in lib.cmr_status_string(99)
-    assert lib.cmr_version() == 20100
+    assert lib.cmr_version() == 20200
     assert lib.cmr_last_rotate_kernel() == b""  # nothing launched on this thread
 
 
@@ -154,6 +155,20 @@ def lib_ok(status):
 def test_positions_rotate_of_nothing_is_a_no_op(lib):
     assert lib.cmr_positions_rotate_qk(None, None, 0, 0, 248078, None, None, None, None, None, 1,
                                        8, 2, 256, 1e7, SEC, 64, None, None) == 0
+    assert lib.cmr_positions_rotate_qk_host(None, None, 0, 0, 248078, None, None, None, None,
+                                            None, 1, 8, 2, 256, 1e7, SEC, 64, None, None) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(theta=0.0), dict(rot_dim=40), dict(head_dim=12),
+                                dict(num_seqs=-1), dict(n=-5), dict(cu=None)])
+def test_positions_rotate_host_rejects_bad_arguments_on_the_host(lib, kw):
+    # refused before anything is enqueued (no GPU needed)
+    a = dict(ids=FAKE, cu=FAKE, num_seqs=2, n=10, theta=1e7, rot_dim=64, head_dim=256)
+    a.update(kw)
+    st = lib.cmr_positions_rotate_qk_host(a["ids"], a["cu"], a["num_seqs"], a["n"], 248078,
+                                          FAKE, FAKE, FAKE, FAKE, FAKE, 1, 8, 2, a["head_dim"],
+                                          a["theta"], SEC, a["rot_dim"], None, None)
+    assert st == cmr.CMR_EINVAL, lib.cmr_last_error_message()
 
 
 @pytest.mark.parametrize("kw", [

@@ -65,6 +65,12 @@ SIGNATURES = {
                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_double, ctypes.POINTER(ctypes.c_int32),
                                                ctypes.c_int32, _i32p, ctypes.c_void_p]),
+    "cmr_positions_rotate_qk_host": (ctypes.c_int, [_i32p, _i32p, ctypes.c_int32, ctypes.c_int64,
+                                               ctypes.c_int32, _i32p, _i32p, _i32p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                               ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                               ctypes.c_double, ctypes.POINTER(ctypes.c_int32),
+                                               ctypes.c_int32, _i32p, ctypes.c_void_p]),
     "cmr_rotate_qk_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                                ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "cmr_rotate_qk_cache_kernel": (ctypes.c_char_p, [ctypes.c_int64, ctypes.c_int32,
@@ -302,11 +308,25 @@ def positions_step(cache_len: torch.Tensor, start: torch.Tensor, amount: torch.T
     return pos
 
 
-def _qk_shapes(q, k, dev, n):
+def _want_pinned(t: torch.Tensor, name: str, dtype: torch.dtype):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.is_cuda or (t.numel() and not t.is_pinned()):
+        raise ValueError(f"{name} must be a pinned (page-locked) CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _qk_shapes(q, k, dev, n, host=False):
     def shape_of(t, name):
         if t is None:
             return None
-        _want(t, name, torch.bfloat16, dev)
+        if host:
+            _want_pinned(t, name, torch.bfloat16)
+        else:
+            _want(t, name, torch.bfloat16, dev)
         if t.dim() == 3:
             return (1,) + tuple(t.shape)
         if t.dim() != 4:
@@ -490,6 +510,50 @@ def positions_rotate_qk(ids: torch.Tensor, cu_seqlens: torch.Tensor, q: Optional
             q.data_ptr() if q is not None and q.numel() else None,
             k.data_ptr() if k is not None and k.numel() else None, L, hq, hk, D, float(theta),
             sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)), "cmr_positions_rotate_qk")
+    return pos, start, amount
+
+
+def positions_rotate_qk_host(ids: torch.Tensor, cu_seqlens: torch.Tensor,
+                             q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                             theta: float = 1e7, sections: Sequence[int] = (11, 11, 10),
+                             rot_dim: int = 64, image_token_id: int = IMAGE_TOKEN_ID,
+                             out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+                             device: Optional[torch.device] = None,
+                             stream: Optional[torch.cuda.Stream] = None):
+    """cmr_positions_rotate_qk_host: the whole path on a batch held in pinned
+    host memory (ids, cu_seqlens, q, k and the outputs are pinned CPU
+    tensors), run by the kernels of `device` (default: the current CUDA
+    device), which read and write those buffers over PCIe.  Asynchronous on
+    `stream` (default: the device's current stream): synchronise it before
+    reading the results or touching the buffers.  Returns (pos [3, N],
+    start [B], amount [B]), pinned."""
+    _want_pinned(ids, "ids", torch.int32)
+    _want_pinned(cu_seqlens, "cu_seqlens", torch.int32)
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+    n, b = ids.numel(), cu_seqlens.numel() - 1
+    if b < 0:
+        raise ValueError("cu_seqlens needs num_seqs + 1 entries")
+    L, hq, hk, D = _qk_shapes(q, k, dev, n, host=True)
+    if out is None:
+        pos = torch.empty((3, n), dtype=torch.int32, pin_memory=True)
+        start = torch.empty(b, dtype=torch.int32, pin_memory=True)
+        amount = torch.empty(b, dtype=torch.int32, pin_memory=True)
+    else:
+        pos, start, amount = out
+        for t, name in ((pos, "pos"), (start, "start"), (amount, "amount")):
+            _want_pinned(t, name, torch.int32)
+        if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
+            raise ValueError("output shapes must be [3, N], [B], [B]")
+    sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
+    with torch.cuda.device(dev):
+        _check(lib().cmr_positions_rotate_qk_host(
+            ids.data_ptr() if n else None, cu_seqlens.data_ptr(), b, n, int(image_token_id),
+            pos.data_ptr() if n else None, start.data_ptr() if b else None,
+            amount.data_ptr() if b else None,
+            q.data_ptr() if q is not None and q.numel() else None,
+            k.data_ptr() if k is not None and k.numel() else None, L, hq, hk, D, float(theta),
+            sec, int(rot_dim), None, _stream_ptr(dev, stream)), "cmr_positions_rotate_qk_host")
     return pos, start, amount
 
 

@@ -49,6 +49,31 @@ cmr_status check_device_ptr(const void* p, const char* name) {
   return CMR_OK;
 }
 
+// Page-locked host memory mapped into the device's address space at the same
+// address (cudaHostAlloc'd or cudaHostRegister'd memory on a system with
+// unified addressing): a kernel reads and writes it directly over PCIe.
+cmr_status check_mapped_host_ptr(const void* p, const char* name) {
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(CMR_EINVAL, "%s: not a CUDA pointer (%s)", name, cudaGetErrorName(e));
+  }
+  if (attr.type != cudaMemoryTypeHost)
+    return fail(CMR_EINVAL, "%s: not page-locked host memory (memory type %d)", name,
+                static_cast<int>(attr.type));
+  if (attr.devicePointer != p)
+    return fail(CMR_EINVAL, "%s: page-locked host memory not mapped at the same address", name);
+  return CMR_OK;
+}
+
+// Where an entry point's buffers live.
+enum class Where { kDevice, kMappedHost };
+
+cmr_status check_ptr(const void* p, const char* name, Where where) {
+  return where == Where::kDevice ? check_device_ptr(p, name) : check_mapped_host_ptr(p, name);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool ranges_overlap(const void* a, const void* b, size_t bytes) {
@@ -61,7 +86,8 @@ bool ranges_overlap(const void* a, const void* b, size_t bytes) {
 // nothing to do.
 cmr_status check_rotate(void* q, void* k, int64_t n_tokens, int32_t num_layers, int32_t hq,
                         int32_t hk, int32_t head_dim, double theta, const int32_t sections[3],
-                        int32_t rot_dim, cmr::RotateArgs* a, cmr::FreqTable* table) {
+                        int32_t rot_dim, cmr::RotateArgs* a, cmr::FreqTable* table,
+                        Where where = Where::kDevice) {
   if (n_tokens < 0 || num_layers < 0) return fail(CMR_EINVAL, "negative n_tokens or num_layers");
   if (hq < 0 || hk < 0 || hq + hk < 1) return fail(CMR_EINVAL, "need hq, hk >= 0, hq + hk >= 1");
   if (head_dim <= 0 || head_dim % 8 != 0) return fail(CMR_EINVAL, "head_dim must be a positive multiple of 8");
@@ -100,8 +126,8 @@ cmr_status check_rotate(void* q, void* k, int64_t n_tokens, int32_t num_layers, 
   if ((hq > 0 && !aligned16(q)) || (hk > 0 && !aligned16(k)))
     return fail(CMR_EINVAL, "q and k must be 16-byte aligned");
   cmr_status s;
-  if (hq > 0 && (s = check_device_ptr(q, "q")) != CMR_OK) return s;
-  if (hk > 0 && (s = check_device_ptr(k, "k")) != CMR_OK) return s;
+  if (hq > 0 && (s = check_ptr(q, "q", where)) != CMR_OK) return s;
+  if (hk > 0 && (s = check_ptr(k, "k", where)) != CMR_OK) return s;
   a->q = static_cast<uint16_t*>(q);
   a->k = static_cast<uint16_t*>(k);
   a->num_layers = num_layers;
@@ -117,7 +143,8 @@ cmr_status check_rotate(void* q, void* k, int64_t n_tokens, int32_t num_layers, 
 // and leaves nothing to do).
 cmr_status check_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                            int64_t n_tokens, const int32_t* out_pos, const int32_t* out_start,
-                           const int32_t* out_amount, const int32_t* device_status) {
+                           const int32_t* out_amount, const int32_t* device_status,
+                           Where where = Where::kDevice) {
   if (num_seqs < 0 || n_tokens < 0) return fail(CMR_EINVAL, "negative num_seqs or n_tokens");
   if (n_tokens > INT32_MAX) return fail(CMR_EINVAL, "n_tokens exceeds int32 indexing");
   if (num_seqs == 0) {
@@ -128,14 +155,17 @@ cmr_status check_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_
     return fail(CMR_EINVAL, "cu_seqlens, out_start and out_amount are required");
   if (n_tokens > 0 && (!ids || !out_pos)) return fail(CMR_EINVAL, "ids and out_pos are required");
   cmr_status s;
-  if ((s = check_device_ptr(cu_seqlens, "cu_seqlens")) != CMR_OK) return s;
-  if ((s = check_device_ptr(out_start, "out_start")) != CMR_OK) return s;
-  if ((s = check_device_ptr(out_amount, "out_amount")) != CMR_OK) return s;
+  if ((s = check_ptr(cu_seqlens, "cu_seqlens", where)) != CMR_OK) return s;
+  if ((s = check_ptr(out_start, "out_start", where)) != CMR_OK) return s;
+  if ((s = check_ptr(out_amount, "out_amount", where)) != CMR_OK) return s;
   if (n_tokens > 0) {
-    if ((s = check_device_ptr(ids, "ids")) != CMR_OK) return s;
-    if ((s = check_device_ptr(out_pos, "out_pos")) != CMR_OK) return s;
+    if ((s = check_ptr(ids, "ids", where)) != CMR_OK) return s;
+    if ((s = check_ptr(out_pos, "out_pos", where)) != CMR_OK) return s;
   }
-  if (device_status && (s = check_device_ptr(device_status, "device_status")) != CMR_OK) return s;
+  // the status word may be device memory or mapped host memory
+  if (device_status && check_device_ptr(device_status, "device_status") != CMR_OK &&
+      (s = check_mapped_host_ptr(device_status, "device_status")) != CMR_OK)
+    return s;
   return CMR_OK;
 }
 
@@ -161,7 +191,7 @@ const char* cmr_last_error_message(void) { return g_message; }
 
 const char* cmr_last_rotate_kernel(void) { return g_last_kernel ? g_last_kernel : ""; }
 
-int32_t cmr_version(void) { return 20100; }  // 2.1.0
+int32_t cmr_version(void) { return 20200; }  // 2.2.0
 
 cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens, int32_t num_seqs,
                          int64_t n_tokens, int32_t image_token_id, int32_t* out_pos,
@@ -356,6 +386,56 @@ cmr_status cmr_positions_rotate_qk(const int32_t* ids, const int32_t* cu_seqlens
   a.pos_out = out_pos;
   a.status = device_status;
   e = cmr::launch_rotate_qk(a, table, st, /*programmatic=*/true);
+  if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
+  return CMR_OK;
+}
+
+cmr_status cmr_positions_rotate_qk_host(const int32_t* ids, const int32_t* cu_seqlens,
+                                        int32_t num_seqs, int64_t n_tokens,
+                                        int32_t image_token_id, int32_t* out_pos,
+                                        int32_t* out_start, int32_t* out_amount, void* q, void* k,
+                                        int32_t num_layers, int32_t hq, int32_t hk,
+                                        int32_t head_dim, double theta,
+                                        const int32_t sections[3], int32_t rot_dim,
+                                        int32_t* device_status, cmr_stream_t stream) {
+  // The checks of cmr_positions_rotate_qk, with every buffer in mapped host
+  // memory (the status word may be either).
+  cmr::RotateArgs a;
+  cmr::FreqTable table;
+  cmr_status s = check_positions(ids, cu_seqlens, num_seqs, n_tokens, out_pos, out_start,
+                                 out_amount, device_status, Where::kMappedHost);
+  if (s != CMR_OK) return s;
+  s = check_rotate(q, k, n_tokens, num_layers, hq, hk, head_dim, theta, sections, rot_dim, &a,
+                   &table, Where::kMappedHost);
+  if (s != CMR_OK) return s;
+  if (num_seqs == 0) return CMR_OK;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (a.n_tokens == 0) {  // no rotation: the planes kernel writes pos
+    cudaError_t e = cmr::launch_positions(ids, cu_seqlens, num_seqs, n_tokens, image_token_id,
+                                          CMR_RULE_CANVAS, nullptr, nullptr, nullptr, out_pos,
+                                          out_start, out_amount, device_status, st);
+    return e == cudaSuccess ? CMR_OK : cuda_fail(e, "positions launch");
+  }
+  // The origin scan reads the ids over PCIe and writes the state; the
+  // row-coalesced kernel (whole rotated parts per instruction, plain loads
+  // and stores: no tensor maps over host memory; the register kernel for
+  // rot_dims it does not take) then derives, writes and uses each token's
+  // planes, moving only the rotated dims of each head row across the bus.
+  cudaError_t e = cmr::launch_positions_origin(ids, cu_seqlens, num_seqs, n_tokens,
+                                               image_token_id, CMR_RULE_CANVAS, nullptr, nullptr,
+                                               nullptr, out_start, out_amount, device_status, st);
+  if (e != cudaSuccess) return cuda_fail(e, "positions launch");
+  a.pos = nullptr;
+  a.cu = cu_seqlens;
+  a.num_seqs = num_seqs;
+  a.pos_offset = nullptr;
+  a.start = out_start;
+  a.amount = out_amount;
+  a.pos_out = out_pos;
+  a.status = device_status;
+  e = cmr::rotate_rows_fits(a) ? cmr::launch_rotate_qk_rows(a, table, st, /*programmatic=*/true)
+                               : cmr::launch_rotate_qk_register(a, table, st,
+                                                                /*programmatic=*/true);
   if (e != cudaSuccess) return cuda_fail(e, "rotate_qk launch");
   return CMR_OK;
 }

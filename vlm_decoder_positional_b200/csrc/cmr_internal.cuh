@@ -120,6 +120,14 @@ cudaError_t launch_positions_step(const int32_t* cache_len, const int32_t* start
 // the staged kernel's Q/K loads start before the wait for pos.
 cudaError_t launch_rotate_qk(const RotateArgs& args, const FreqTable& table, cudaStream_t stream,
                              bool programmatic = false);
+// The register kernel alone (plain loads and stores, no tensor maps).
+cudaError_t launch_rotate_qk_register(const RotateArgs& args, const FreqTable& table,
+                                      cudaStream_t stream, bool programmatic = false);
+// The row-coalesced kernel for Q/K in mapped host memory (rotate_rows.cu):
+// shift-state planes only; rot_dim / 8 must divide 32.
+bool rotate_rows_fits(const RotateArgs& args);
+cudaError_t launch_rotate_qk_rows(const RotateArgs& args, const FreqTable& table,
+                                  cudaStream_t stream, bool programmatic = false);
 
 // TMA tensor map of a bf16 tensor: dims[0] is contiguous, strides_bytes[i] is
 // the byte stride of dims[i + 1] (any order), box[i] the box extent per dim.

@@ -252,6 +252,11 @@ cudaError_t launch_rotate_qk(const RotateArgs& in, const FreqTable& table, cudaS
     const cudaError_t e = launch_rotate_qk_staged(in, table, stream, programmatic, &launched);
     if (e != cudaSuccess || launched) return e;
   }
+  return launch_rotate_qk_register(in, table, stream, programmatic);
+}
+
+cudaError_t launch_rotate_qk_register(const RotateArgs& in, const FreqTable& table,
+                                      cudaStream_t stream, bool programmatic) {
   RotateArgs a = in;
   const bool from_shift = a.pos == nullptr;
   const int64_t items_per_cta = kThreads / a.units_per_head;
