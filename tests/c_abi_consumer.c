@@ -6,7 +6,10 @@
  *                         index 6, in cudaMalloc'd buffers; prints "p T H W"
  *                         lines and "start amount" for the test to compare,
  *                         then "frames same" if the multi-frame entry point
- *                         without a workspace gives the same planes */
+ *                         without a workspace gives the same planes, and
+ *                         "host batch same" if the whole path on a batch in
+ *                         cudaHostAlloc'd memory gives the device path's
+ *                         planes, state and rotated Q/K bytes */
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -53,6 +56,8 @@ static int host_checks(void) {
                                 256, 1e7, bad_sections, 64, NULL, NULL) == CMR_EINVAL);
   /* several frames per prompt: the workspace size and the host checks */
   CHECK(cmr_positions_frames_workspace_bytes(32, 32 * 8192) == 16u * 32 * 2);
+  CHECK(cmr_positions_rotate_qk_host(NULL, NULL, 0, 0, 248078, NULL, NULL, NULL, NULL, NULL, 1,
+                                     8, 2, 256, 1e7, sections, 64, NULL, NULL) == CMR_OK);
   CHECK(cmr_positions_frames(fake, fake, 1, 10, 248078, 0, fake, fake, fake, fake, 1 << 20, NULL,
                              NULL) == CMR_EINVAL);
   CHECK(cmr_positions_frames_noalloc(fake, fake, 16385, 16385, 248078, 8, fake, fake, fake, NULL,
@@ -68,6 +73,9 @@ extern cuda_err cudaMalloc(void** p, size_t bytes);
 extern cuda_err cudaFree(void* p);
 extern cuda_err cudaMemcpy(void* dst, const void* src, size_t bytes, int kind);
 extern cuda_err cudaDeviceSynchronize(void);
+extern cuda_err cudaHostAlloc(void** p, size_t bytes, unsigned int flags);
+extern cuda_err cudaFreeHost(void* p);
+#define HOST_ALLOC_MAPPED 2u /* cudaHostAllocMapped */
 
 static int device_run(void) {
   enum { N = 80, O = 6 };
@@ -110,6 +118,66 @@ static int device_run(void) {
   int32_t pos2[3 * N];
   CHECK(cudaMemcpy(pos2, d_pos2, sizeof pos2, 2) == 0);
   if (memcmp(pos, pos2, sizeof pos) == 0) printf("frames same\n");
+  /* the whole path on a batch in mapped page-locked host memory, against the
+     same call on device copies */
+  {
+    enum { HQ = 8, HK = 2, D = 256 };
+    const int32_t sections[3] = {11, 11, 10};
+    const size_t qn = (size_t)N * HQ * D, kn = (size_t)N * HK * D;
+    int32_t *h_ids, *h_cu, *h_pos, *h_start, *h_amount;
+    uint16_t *h_q, *h_k, *d_q, *d_k;
+    CHECK(cudaHostAlloc((void**)&h_ids, sizeof ids, HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_cu, sizeof cu, HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_pos, 3 * N * sizeof(int32_t), HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_start, sizeof(int32_t), HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_amount, sizeof(int32_t), HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_q, qn * 2, HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaHostAlloc((void**)&h_k, kn * 2, HOST_ALLOC_MAPPED) == 0);
+    CHECK(cudaMalloc((void**)&d_q, qn * 2) == 0);
+    CHECK(cudaMalloc((void**)&d_k, kn * 2) == 0);
+    memcpy(h_ids, ids, sizeof ids);
+    memcpy(h_cu, cu, sizeof cu);
+    /* bf16 values of magnitude 0.5 .. 2 with both signs, from a fixed LCG */
+    uint32_t r = 12345u;
+    for (size_t i = 0; i < qn; ++i) { r = r * 1664525u + 1013904223u; h_q[i] = (uint16_t)(0x3f00u + (r >> 25) + ((r >> 24) & 1u) * 0x8000u); }
+    for (size_t i = 0; i < kn; ++i) { r = r * 1664525u + 1013904223u; h_k[i] = (uint16_t)(0x3f00u + (r >> 25) + ((r >> 24) & 1u) * 0x8000u); }
+    CHECK(cudaMemcpy(d_q, h_q, qn * 2, 1) == 0);
+    CHECK(cudaMemcpy(d_k, h_k, kn * 2, 1) == 0);
+    s = cmr_positions_rotate_qk(d_ids, d_cu, 1, N, 248078, d_pos, d_start, d_amount, d_q, d_k, 1,
+                                HQ, HK, D, 1e7, sections, 64, NULL, NULL);
+    if (s != CMR_OK) {
+      fprintf(stderr, "cmr_positions_rotate_qk: %s\n", cmr_last_error_message());
+      return 1;
+    }
+    s = cmr_positions_rotate_qk_host(h_ids, h_cu, 1, N, 248078, h_pos, h_start, h_amount, h_q,
+                                     h_k, 1, HQ, HK, D, 1e7, sections, 64, NULL, NULL);
+    if (s != CMR_OK) {
+      fprintf(stderr, "cmr_positions_rotate_qk_host: %s\n", cmr_last_error_message());
+      return 1;
+    }
+    CHECK(cudaDeviceSynchronize() == 0);
+    uint16_t* q_dev = malloc(qn * 2);
+    uint16_t* k_dev = malloc(kn * 2);
+    CHECK(q_dev && k_dev);
+    CHECK(cudaMemcpy(q_dev, d_q, qn * 2, 2) == 0);
+    CHECK(cudaMemcpy(k_dev, d_k, kn * 2, 2) == 0);
+    CHECK(cudaMemcpy(pos2, d_pos, sizeof pos2, 2) == 0);
+    if (memcmp(h_pos, pos2, sizeof pos2) == 0 && memcmp(h_pos, pos, sizeof pos) == 0 &&
+        *h_start == start && *h_amount == amount && memcmp(h_q, q_dev, qn * 2) == 0 &&
+        memcmp(h_k, k_dev, kn * 2) == 0)
+      printf("host batch same\n");
+    free(q_dev);
+    free(k_dev);
+    cudaFreeHost(h_ids);
+    cudaFreeHost(h_cu);
+    cudaFreeHost(h_pos);
+    cudaFreeHost(h_start);
+    cudaFreeHost(h_amount);
+    cudaFreeHost(h_q);
+    cudaFreeHost(h_k);
+    cudaFree(d_q);
+    cudaFree(d_k);
+  }
   cudaFree(d_pos2);
   cudaFree(d_ids);
   cudaFree(d_cu);

@@ -1,7 +1,8 @@
 """A plain C11 program uses the C ABI directly: the header compiles as C with
 -Wall -Werror, the host checks answer without a GPU, and on a GPU the planes
 of the 80-token prompt with <image> at 6 equal the golden table, also through
-the multi-frame entry point that allocates nothing."""
+the multi-frame entry point that allocates nothing, and the whole path on a
+batch in cudaHostAlloc'd memory equals the device path byte for byte."""
 import os
 import subprocess
 
@@ -42,3 +43,4 @@ def test_c_consumer_device_planes(consumer):
     assert got == want
     assert lines[80].split() == ["73", "58"]
     assert lines[81] == "frames same"
+    assert lines[82] == "host batch same"
