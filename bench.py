@@ -547,10 +547,11 @@ def run_ours(args):
         e2e = {"skipped": f"--op {args.op} times the device step only; the end-to-end path "
                           "is measured with --op rotate"}
 
+    # the two ceilings of an HBM-bound launch (the staged kernel's batches are
+    # larger than L2; the small workloads are bound by launch latency)
     ceiling = same_size_copy = None
     if args.op == "rotate" and kernel_ran == "rotate_qk_staged_kernel":
         ceiling = run_copy_pattern_probe(wl, dev, stream)
-    if args.op == "rotate":
         same_size_copy = run_plain_copy_probe(rot_b, dev, stream)
 
     if rank == 0:
