@@ -21,7 +21,9 @@
 //   1. frames_summary_kernel reduces its slice's tokens to that 16-byte
 //      summary in a caller-provided workspace [num_seqs][slices], with the
 //      ids of kFrSumUnroll block steps in flight before it folds any;
-//   2. frames_positions_kernel, launched programmatically behind it, loads its
+//   2. frames_positions_kernel, launched programmatically behind it, walks
+//      the slices in the reverse of the summary kernel's order (the ids that
+//      kernel read last are the likeliest to be in L2 still), loads its
 //      first ids before it waits for the summaries, has one warp fold the
 //      summaries of the slices before its own into a carry, then walks its
 //      slice in chunks of kFrThreads x kFrItems tokens: each thread folds its
@@ -177,11 +179,10 @@ struct FrSlice {
   int32_t len, p0, p1;
 };
 
-// Prompt blockIdx.x of the batch: false (and *bad set) when its cu_seqlens
-// entries are malformed.
+// Prompt b of the batch: false (and *bad set) when its cu_seqlens entries
+// are malformed.
 __device__ __forceinline__ bool fr_prompt(const int32_t* __restrict__ cu, int32_t num_seqs,
-                                          int64_t n_tokens, bool* bad, FrSlice* sl) {
-  const int32_t b = blockIdx.x;
+                                          int64_t n_tokens, int32_t b, bool* bad, FrSlice* sl) {
   const int64_t first = __ldg(cu + b);
   const int64_t last = __ldg(cu + b + 1);
   *bad = first < 0 || last < first || last > n_tokens || (b == 0 && first != 0) ||
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kFrThreads)
   pdl::launch_dependents();
   bool bad;
   FrSlice sl;
-  if (!fr_prompt(cu, num_seqs, n_tokens, &bad, &sl)) {
+  if (!fr_prompt(cu, num_seqs, n_tokens, blockIdx.x, &bad, &sl)) {
     if (bad && blockIdx.y == 0 && threadIdx.x == 0 && status != nullptr)
       atomicOr(status, CMR_DEVICE_BAD_CU_SEQLENS);
     return;
@@ -306,11 +307,14 @@ __global__ void __launch_bounds__(kFrThreads, kFrPosBlocks)
   int turn = 0;
   bool bad;
   FrSlice sl;
-  if (!fr_prompt(cu, num_seqs, n_tokens, &bad, &sl)) return;
-  fr_range(blockIdx.y, gridDim.y, &sl);
+  // slices in the reverse of the summary kernel's order: the ids it read last
+  // are the likeliest to be in L2 still
+  const uint32_t bx = gridDim.x - 1 - blockIdx.x, by = gridDim.y - 1 - blockIdx.y;
+  if (!fr_prompt(cu, num_seqs, n_tokens, static_cast<int32_t>(bx), &bad, &sl)) return;
+  fr_range(by, gridDim.y, &sl);
   // The CTA holding the prompt's last token (slice 0 of an empty prompt)
   // ends with the summary of the whole prompt and writes its state.
-  const bool writer = sl.len == 0 ? blockIdx.y == 0 : (sl.p0 < sl.p1 && sl.p1 == sl.len);
+  const bool writer = sl.len == 0 ? by == 0 : (sl.p0 < sl.p1 && sl.p1 == sl.len);
   if (sl.p0 >= sl.p1 && !writer) return;
   const int32_t frame_len = side * side + 3;
   const int64_t lo = sl.first + sl.p0, hi = sl.first + sl.p1;
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kFrThreads, kFrPosBlocks)
   // warps read the carry after the first block scan's barrier
   if (threadIdx.x < 32) {
     const Summary before =
-        warp_fold(work + static_cast<int64_t>(blockIdx.x) * gridDim.y, blockIdx.y, frame_len);
+        warp_fold(work + static_cast<int64_t>(bx) * gridDim.y, by, frame_len);
     if (threadIdx.x == 0) s_carry = before;
   }
   Summary carry{0, 0, 0, 0};  // the prompt's summary up to the current chunk
@@ -423,14 +427,14 @@ __global__ void __launch_bounds__(kFrThreads, kFrPosBlocks)
   if (writer && threadIdx.x == 0) {
     // an empty prompt ran no chunk: its carry is slice 0's, the identity
     if (carry.n == 0) {
-      out_start[blockIdx.x] = kTextOnlyStart;
-      out_amount[blockIdx.x] = 0;
+      out_start[bx] = kTextOnlyStart;
+      out_amount[bx] = 0;
     } else {
       const int64_t span = side + 1;
       const int64_t start = static_cast<int64_t>(carry.last) + frame_len;
       const int64_t anchor = carry.first + static_cast<int64_t>(carry.n - 1) * span + carry.gaps;
-      out_start[blockIdx.x] = static_cast<int32_t>(start);
-      out_amount[blockIdx.x] = static_cast<int32_t>(start - (anchor + span));
+      out_start[bx] = static_cast<int32_t>(start);
+      out_amount[bx] = static_cast<int32_t>(start - (anchor + span));
     }
   }
 }
