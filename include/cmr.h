@@ -14,7 +14,9 @@
  * Conventions for every entry point:
  *   - Pointers named "device" must point to memory the current CUDA device can
  *     read/write (cudaMalloc, torch CUDA tensors, managed memory).  Host
- *     pointers are rejected with CMR_EINVAL where the runtime can tell.
+ *     pointers are rejected with CMR_EINVAL where the runtime can tell.  The
+ *     one exception, cmr_positions_rotate_qk_host, takes mapped page-locked
+ *     host memory instead (and rejects device memory).
  *   - The caller owns every buffer.  The library never allocates, frees or
  *     synchronises; all work is enqueued on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream) and runs asynchronously.
