@@ -158,6 +158,43 @@ def test_cluster_scan_in_chunks_and_the_one_call_path(cuda_device):
         np.testing.assert_array_equal(g.cpu().numpy(), w)
 
 
+CAPTURE_FIRST = r"""
+import sys
+import numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import oracle
+from vlm_decoder_positional_b200 import cmr, inputs
+dev = torch.device("cuda", 0)
+rng = np.random.default_rng(40)
+ids_np, cu_np = inputs.pack([inputs.prompt_ids(rng, 300_000, o) for o in (-1, 250_000)])
+ids, cu = torch.from_numpy(ids_np).to(dev), torch.from_numpy(cu_np).to(dev)
+pos = torch.empty((3, ids.numel()), dtype=torch.int32, device=dev)
+st = torch.empty(2, dtype=torch.int32, device=dev)
+am = torch.empty(2, dtype=torch.int32, device=dev)
+g = torch.cuda.CUDAGraph()
+with torch.cuda.graph(g):  # the library's first launch in this process
+    cmr.positions(ids, cu, out=(pos, st, am))
+g.replay()
+torch.cuda.synchronize()
+want = oracle.positions(ids_np, cu_np, inputs.IMAGE_TOKEN_ID)
+for a, b in zip((pos, st, am), want):
+    np.testing.assert_array_equal(a.cpu().numpy(), b)
+print("ok")
+"""
+
+
+def test_cluster_scan_first_launched_inside_a_graph_capture(cuda_device):
+    # the occupancy query that picks the cluster form runs during the capture
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", CAPTURE_FIRST, root], capture_output=True,
+                         text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert out.stdout.strip().endswith("ok")
+
+
 def test_many_short_prompts_and_repeated_markers(cuda_device):
     rng = np.random.default_rng(4)
     lens = rng.integers(0, 90, size=5000)

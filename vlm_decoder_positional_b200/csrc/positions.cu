@@ -27,6 +27,7 @@
 #include <cooperative_groups.h>
 
 #include <climits>
+#include <mutex>
 
 #include "canvas.cuh"
 #include "pdl.cuh"
@@ -259,6 +260,32 @@ __global__ void canvas_positions_step_kernel(const int32_t* __restrict__ cache_l
   }
 }
 
+// Whether the current device can hold at least one cluster of k origin CTAs
+// (occupancy query, no launch; cached per device and k).
+bool origin_clusters_fit(int k, const cudaLaunchConfig_t& cfg) {
+  static std::mutex mu;
+  static int8_t known[64][kOriginMaxCluster + 1] = {};  // 0 unknown, 1 fits, -1 does not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  int8_t& state = known[dev][k];
+  if (state == 0) {
+    cudaLaunchConfig_t one = cfg;
+    one.gridDim = dim3(static_cast<unsigned>(k));
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, canvas_origin_kernel<true>, &one) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return false;  // not cached: the next call asks again
+    }
+    state = clusters > 0 ? 1 : -1;
+  }
+  return state > 0;
+}
+
 }  // namespace
 
 cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlens,
@@ -290,6 +317,14 @@ cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlen
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (!origin_clusters_fit(k, cfg)) {
+    // a device (or a share of one) that cannot place such clusters: one CTA
+    // per chunk gives the same results
+    canvas_origin_kernel<false><<<static_cast<unsigned>(num_seqs), kOriginThreads, 0, stream>>>(
+        ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule, pos_offset, in_start,
+        in_amount, out_start, out_amount, device_status);
+    return cudaGetLastError();
+  }
   return cudaLaunchKernelEx(&cfg, canvas_origin_kernel<true>, ids, cu_seqlens, num_seqs,
                             n_tokens, image_token_id, rule, pos_offset, in_start, in_amount,
                             out_start, out_amount, device_status);
