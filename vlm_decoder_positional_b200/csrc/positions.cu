@@ -131,7 +131,9 @@ __device__ __forceinline__ int64_t first_marker_cluster(const int32_t* __restric
       if (q == 0) *s_all = all;
     }
     __syncthreads();
-    const int all = *s_all;  // rewritten only after the next round's block barriers
+    // warp 0 rewrites s_all only after the next round's cluster barrier, which
+    // every thread of the CTA reaches after this read
+    const int all = *s_all;
     if (all != INT_MAX) {
       result = all;
       break;
