@@ -614,24 +614,26 @@ def probe_lib():
     from vlm_decoder_positional_b200 import build as libbuild
     libbuild.build()
     lib = ctypes.CDLL(libbuild.PROBE_LIB)
-    f = lib.cmr_probe_copy_pattern
+    f = lib.cmr_probe_copy_pattern_tiles
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
-                  ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
-                  ctypes.c_void_p]
+                  ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_void_p, ctypes.c_void_p]
     return f
 
 
-def run_copy_pattern_probe(wl, dev, stream, launches=10, warmup=3):
+def run_copy_pattern_probe(wl, dev, stream, launches=10, warmup=3, tiles_per_cta=1):
     """The ceiling of the staged rotation's access pattern: copy_pattern_kernel
     moves the same rotated dims of Q and K through the same TMA staging with no
     math (an identity copy), timed like the rotate launch (CUDA events around
-    each of `launches` launches).  Returns GB/s over the Q/K bytes it moves."""
+    each of `launches` launches).  tiles_per_cta > 1: each CTA walks that many
+    consecutive tiles through one ring.  Returns GB/s over the Q/K bytes it
+    moves."""
     f = probe_lib()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     n = wl.q.shape[1]
     args = (wl.q.data_ptr(), wl.k.data_ptr(), n, wl.num_layers, wl.hq, wl.hk, wl.head_dim,
-            status.data_ptr(), stream.cuda_stream)
+            int(tiles_per_cta), status.data_ptr(), stream.cuda_stream)
     for _ in range(warmup):
         if f(*args) != 0:
             raise RuntimeError("copy-pattern probe: launch refused")
@@ -685,11 +687,17 @@ def run_probe_only(args):
     torch.cuda.set_device(dev)
     wl = inputs.make_config(args.workload, device=dev)
     stream = torch.cuda.current_stream(dev)
-    res = run_copy_pattern_probe(wl, dev, stream, launches=args.steps, warmup=args.warmup)
+    if args.layers is not None:
+        wl.num_layers = args.layers
+        wl.q = inputs.random_qk((args.layers, wl.n_tokens, wl.hq, wl.head_dim), 11, dev)
+        wl.k = inputs.random_qk((args.layers, wl.n_tokens, wl.hk, wl.head_dim), 12, dev)
+    res = run_copy_pattern_probe(wl, dev, stream, launches=args.steps, warmup=args.warmup,
+                                 tiles_per_cta=args.tiles_per_cta)
     plain = run_plain_copy_probe(res["bytes"], dev, stream, launches=args.steps,
                                  warmup=args.warmup)
     peak, src = measured_peak()
     print(json.dumps({"probe": "copy-pattern", "workload": workload_label(wl),
+                      "tiles_per_cta": args.tiles_per_cta, "layers": wl.num_layers,
                       "gbs": res["gbs"], "ms_per_launch": res["ms"], "bytes": res["bytes"],
                       "peak": peak, "peak_source": src, "frac_of_peak": res["gbs"] / peak,
                       "launches": args.steps, "what": res["what"],
@@ -997,6 +1005,9 @@ def main():
                          "launch timed on its own")
     ap.add_argument("--probe", choices=["copy-pattern"], default=None,
                     help="run only the copy-pattern ceiling probe (--steps launches)")
+    ap.add_argument("--tiles-per-cta", type=int, default=1,
+                    help="--probe copy-pattern: consecutive 8-token tiles per CTA (1: the "
+                         "rotation's staging)")
     ap.add_argument("--launch", choices=["graph", "eager"], default="graph",
                     help="graph: replay a captured CUDA graph per call (default); eager: "
                          "launch through the Python binding every step")

@@ -4,7 +4,9 @@
 // heads through the same ring of stages -- with no cos/sin and no rotation:
 // each box is stored back unchanged.  Its rate is what this access pattern
 // can reach on the device, the ceiling the rotation is judged against beside
-// the plain-copy peak.  It leaves Q and K bit for bit as they were.
+// the plain-copy peak.  It leaves Q and K bit for bit as they were.  With
+// tiles_per_cta > 1 each CTA walks that many consecutive tiles through one
+// ring, the staging the rotation measured and did not keep.
 //
 // A measurement aid, not part of the library: it is built into its own
 // libcmr_probe.so and is called only by the benchmark.
@@ -28,6 +30,8 @@ struct ProbeArgs {
   int32_t num_layers, hq, hk;
   uint32_t q_box_bytes, stage_bytes;
   int32_t stages;
+  int32_t tiles_per_cta;  // 1 as the rotation; more: a CTA walks consecutive tiles
+  int64_t tiles;          // 8-token tiles in the batch
   int32_t* status;
 };
 
@@ -49,12 +53,19 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   const int L = args.num_layers;
-  const int t0 = static_cast<int>(blockIdx.x) * kTileTokens;
+  // item i = (tile first + i / L, layer i % L); one tile per CTA in the
+  // rotation's own staging, several with tiles_per_cta > 1
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * args.tiles_per_cta;
+  const int64_t my_tiles =
+      args.tiles - first < args.tiles_per_cta ? args.tiles - first : args.tiles_per_cta;
+  const int items = static_cast<int>(my_tiles) * L;
   if (threadIdx.x >= 32) {
     if (threadIdx.x != 32) return;
     int issued = 0, s = 0;
     uint32_t phase = 0;
-    for (int l = 0; l < L; ++l) {
+    for (int i = 0; i < items; ++i) {
+      const int l = i % L;
+      const int t0 = static_cast<int>((first + i / L) * kTileTokens);
       if (!cmr::tma::mbar_wait(empty0 + 8 * s, phase ^ 1u)) {
         if (args.status) atomicOr(args.status, 4);
         break;
@@ -78,7 +89,9 @@ __global__ void __launch_bounds__(kThreads)
   }
   int st = 0, prev = S - 1;
   uint32_t phase = 0;
-  for (int l = 0; l < L; ++l) {
+  for (int i = 0; i < items; ++i) {
+    const int l = i % L;
+    const int t0 = static_cast<int>((first + i / L) * kTileTokens);
     const bool landed = cmr::tma::mbar_wait(full0 + 8 * st, phase);
     if (cmr::tma::named_any(1, 32, !landed)) {
       if (threadIdx.x == 0 && args.status) atomicOr(args.status, 4);
@@ -90,7 +103,7 @@ __global__ void __launch_bounds__(kThreads)
       if (args.hk > 0) cmr::tma::store_4d(&k_map, src + args.q_box_bytes, 0, t0, 0, l);
       cmr::tma::bulk_commit();
       cmr::tma::bulk_wait_read<1>();
-      if (l > 0) cmr::tma::mbar_arrive(empty0 + 8 * prev);
+      if (i > 0) cmr::tma::mbar_arrive(empty0 + 8 * prev);
     }
     __syncwarp();
     prev = st;
@@ -142,14 +155,18 @@ bool encode(CUtensorMap* map, void* base, int64_t n, int heads, int layers, int 
 
 // Copies the first 64 dims of every head row of q [L, N, hq, head_dim] and
 // k [L, N, hk, head_dim] (bf16, device, 16-byte aligned) onto themselves
-// through the staged path.  Returns 0 when enqueued, 1 for arguments it does
-// not take, 2 for a CUDA error.  status (optional, device int32) gets bit 4
-// if a bounded wait gave up.
-extern "C" __attribute__((visibility("default"))) int cmr_probe_copy_pattern(
+// through the staged path, each CTA walking tiles_per_cta consecutive 8-token
+// tiles (1: the rotation's own staging; more: the form that overlaps one
+// tile's loads with the previous tile's work inside a CTA, through a ring of
+// min(3, tiles_per_cta x layers) stages).  Returns 0 when enqueued, 1 for
+// arguments it does not take, 2 for a CUDA error.  status (optional, device
+// int32) gets bit 4 if a bounded wait gave up.
+extern "C" __attribute__((visibility("default"))) int cmr_probe_copy_pattern_tiles(
     void* q, void* k, int64_t n_tokens, int32_t num_layers, int32_t hq, int32_t hk,
-    int32_t head_dim, int32_t* status, cudaStream_t stream) {
+    int32_t head_dim, int32_t tiles_per_cta, int32_t* status, cudaStream_t stream) {
   if (n_tokens <= 0 || num_layers <= 0 || hq < 0 || hk < 0 || hq + hk < 1 || head_dim < 64 ||
-      head_dim % 8 != 0 || (hq > 0 && !q) || (hk > 0 && !k) ||
+      head_dim % 8 != 0 || (hq > 0 && !q) || (hk > 0 && !k) || tiles_per_cta < 1 ||
+      tiles_per_cta > 64 ||
       (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k)) % 16 != 0)
     return 1;
   CUtensorMap q_map{}, k_map{};
@@ -161,11 +178,22 @@ extern "C" __attribute__((visibility("default"))) int cmr_probe_copy_pattern(
   a.hk = hk;
   a.q_box_bytes = kRowBytes * kTileTokens * hq;
   a.stage_bytes = a.q_box_bytes + kRowBytes * kTileTokens * hk;
-  a.stages = num_layers < kStages ? num_layers : kStages;
+  const int64_t items = static_cast<int64_t>(num_layers) * tiles_per_cta;
+  a.stages = items < kStages ? static_cast<int32_t>(items) : kStages;
+  a.tiles_per_cta = tiles_per_cta;
+  a.tiles = (n_tokens + kTileTokens - 1) / kTileTokens;
   a.status = status;
   const size_t smem = 1024 + static_cast<size_t>(a.stages) * (a.stage_bytes + 16);
   if (smem > 48 * 1024) return 1;  // the probe serves the ring sizes of 8 + 2 heads
-  const int64_t tiles = (n_tokens + kTileTokens - 1) / kTileTokens;
-  copy_pattern_kernel<<<static_cast<unsigned>(tiles), kThreads, smem, stream>>>(q_map, k_map, a);
+  const int64_t ctas = (a.tiles + tiles_per_cta - 1) / tiles_per_cta;
+  copy_pattern_kernel<<<static_cast<unsigned>(ctas), kThreads, smem, stream>>>(q_map, k_map, a);
   return cudaGetLastError() == cudaSuccess ? 0 : 2;
+}
+
+// cmr_probe_copy_pattern_tiles with one tile per CTA: the rotation's staging.
+extern "C" __attribute__((visibility("default"))) int cmr_probe_copy_pattern(
+    void* q, void* k, int64_t n_tokens, int32_t num_layers, int32_t hq, int32_t hk,
+    int32_t head_dim, int32_t* status, cudaStream_t stream) {
+  return cmr_probe_copy_pattern_tiles(q, k, n_tokens, num_layers, hq, hk, head_dim, 1, status,
+                                      stream);
 }
