@@ -136,3 +136,28 @@ def test_device_and_pageable_buffers_are_refused(cuda_device):
     with pytest.raises(ValueError):
         cmr.positions_rotate_qk_host(torch.from_numpy(wl.ids), pinned(wl.cu_seqlens),
                                      host["q"], host["k"], device=dev)
+
+
+def test_malformed_cu_seqlens_sets_a_host_status_word(cuda_device):
+    # the status word may itself live in mapped host memory
+    dev = cuda_device
+    n = 100
+    ids = pinned(np.zeros(n, np.int32))
+    q = pinned(inputs.random_qk((1, n, 8, 256), 5, "cpu"))
+    k = pinned(inputs.random_qk((1, n, 2, 256), 6, "cpu"))
+    sec = (__import__("ctypes").c_int32 * 3)(11, 11, 10)
+    for bad in ([0, 60, 50, 100], [0, 50, 120], [5, 50, 100]):
+        cu = pinned(np.array(bad, np.int32))
+        b = len(bad) - 1
+        pos = pinned(torch.empty((3, n), dtype=torch.int32))
+        st = pinned(torch.empty(b, dtype=torch.int32))
+        am = pinned(torch.empty(b, dtype=torch.int32))
+        status = pinned(torch.zeros(1, dtype=torch.int32))
+        with torch.cuda.device(dev):
+            rc = cmr.lib().cmr_positions_rotate_qk_host(
+                ids.data_ptr(), cu.data_ptr(), b, n, inputs.IMAGE_TOKEN_ID, pos.data_ptr(),
+                st.data_ptr(), am.data_ptr(), q.data_ptr(), k.data_ptr(), 1, 8, 2, 256, 1e7, sec,
+                64, status.data_ptr(), None)
+        assert rc == cmr.CMR_OK, cmr.lib().cmr_last_error_message()
+        torch.cuda.synchronize(dev)
+        assert int(status[0]) & cmr.CMR_DEVICE_BAD_CU_SEQLENS, bad
