@@ -76,9 +76,12 @@ def test_host_batch_against_the_oracle(cuda_device):
     q_in = wl.q.view(torch.int16).numpy().view(np.uint16).copy()
     k_in = wl.k.view(torch.int16).numpy().view(np.uint16).copy()
     q_h, k_h = pinned(wl.q), pinned(wl.k)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
     pos, start, amount = cmr.positions_rotate_qk_host(pinned(wl.ids), pinned(wl.cu_seqlens),
-                                                      q_h, k_h, device=dev)
+                                                      q_h, k_h, device=dev,
+                                                      device_status=status)
     torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0
     want = oracle.positions(wl.ids, wl.cu_seqlens, inputs.IMAGE_TOKEN_ID)
     for g, w in zip((pos, start, amount), want):
         np.testing.assert_array_equal(g.numpy(), w)

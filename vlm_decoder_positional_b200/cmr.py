@@ -519,13 +519,15 @@ def positions_rotate_qk_host(ids: torch.Tensor, cu_seqlens: torch.Tensor,
                              rot_dim: int = 64, image_token_id: int = IMAGE_TOKEN_ID,
                              out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
                              device: Optional[torch.device] = None,
-                             stream: Optional[torch.cuda.Stream] = None):
+                             stream: Optional[torch.cuda.Stream] = None,
+                             device_status: Optional[torch.Tensor] = None):
     """cmr_positions_rotate_qk_host: the whole path on a batch held in pinned
     host memory (ids, cu_seqlens, q, k and the outputs are pinned CPU
     tensors), run by the kernels of `device` (default: the current CUDA
     device), which read and write those buffers over PCIe.  Asynchronous on
     `stream` (default: the device's current stream): synchronise it before
-    reading the results or touching the buffers.  Returns (pos [3, N],
+    reading the results or touching the buffers.  device_status: an int32
+    [1] tensor on that device or pinned on the host.  Returns (pos [3, N],
     start [B], amount [B]), pinned."""
     _want_pinned(ids, "ids", torch.int32)
     _want_pinned(cu_seqlens, "cu_seqlens", torch.int32)
@@ -545,6 +547,13 @@ def positions_rotate_qk_host(ids: torch.Tensor, cu_seqlens: torch.Tensor,
             _want_pinned(t, name, torch.int32)
         if pos.shape != (3, n) or start.numel() != b or amount.numel() != b:
             raise ValueError("output shapes must be [3, N], [B], [B]")
+    if device_status is None:
+        st_ptr = None
+    elif device_status.is_cuda:
+        st_ptr = _status_ptr(device_status, dev)
+    else:
+        _want_pinned(device_status, "device_status", torch.int32)
+        st_ptr = device_status.data_ptr()
     sec = (ctypes.c_int32 * 3)(*[int(v) for v in sections])
     with torch.cuda.device(dev):
         _check(lib().cmr_positions_rotate_qk_host(
@@ -553,7 +562,7 @@ def positions_rotate_qk_host(ids: torch.Tensor, cu_seqlens: torch.Tensor,
             amount.data_ptr() if b else None,
             q.data_ptr() if q is not None and q.numel() else None,
             k.data_ptr() if k is not None and k.numel() else None, L, hq, hk, D, float(theta),
-            sec, int(rot_dim), None, _stream_ptr(dev, stream)), "cmr_positions_rotate_qk_host")
+            sec, int(rot_dim), st_ptr, _stream_ptr(dev, stream)), "cmr_positions_rotate_qk_host")
     return pos, start, amount
 
 
