@@ -96,7 +96,7 @@ typedef enum cmr_status {
  *                and write no planes for the prompts whose bounds are invalid
  *                (their out_start / out_amount entries are then unspecified).
  *                The library never clears it.
- * Two kernels: one CTA per prompt (a cluster of up to 8 CTAs when prompts
+ * Two kernels: one CTA per prompt (a cluster of up to 16 CTAs when prompts
  * average more than 65,536 tokens) scans its ids up to the first marker (no
  * id is read twice) and writes the state; then CTAs over slices of about
  * 2,048 tokens write the planes, reading the state back from out_start /

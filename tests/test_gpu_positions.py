@@ -100,7 +100,7 @@ BLOCK = 16_384  # ids per block of the origin scan
 @pytest.mark.parametrize("length", [120_000, 200_000, 300_000, 1_000_000])
 def test_cluster_scan_block_and_rank_boundaries(cuda_device, length):
     # prompts this long average more than four blocks of ids, so each one is
-    # scanned by a cluster of 2, 4 or 8 CTAs dealing the blocks round-robin;
+    # scanned by a cluster of 2, 4, 8 or 16 CTAs dealing the blocks round-robin;
     # markers sit on both sides of every block edge the prompt has (so on
     # every rank and round), first and last, or nowhere
     rng = np.random.default_rng(10 + length // 1000)
@@ -166,7 +166,8 @@ import oracle
 from vlm_decoder_positional_b200 import cmr, inputs
 dev = torch.device("cuda", 0)
 rng = np.random.default_rng(40)
-ids_np, cu_np = inputs.pack([inputs.prompt_ids(rng, 300_000, o) for o in (-1, 250_000)])
+n = int(sys.argv[2])
+ids_np, cu_np = inputs.pack([inputs.prompt_ids(rng, n, o) for o in (-1, n - 50_000)])
 ids, cu = torch.from_numpy(ids_np).to(dev), torch.from_numpy(cu_np).to(dev)
 pos = torch.empty((3, ids.numel()), dtype=torch.int32, device=dev)
 st = torch.empty(2, dtype=torch.int32, device=dev)
@@ -183,14 +184,16 @@ print("ok")
 """
 
 
-def test_cluster_scan_first_launched_inside_a_graph_capture(cuda_device):
-    # the occupancy query that picks the cluster form runs during the capture
+@pytest.mark.parametrize("length", [300_000, 1_000_000])
+def test_cluster_scan_first_launched_inside_a_graph_capture(cuda_device, length):
+    # the occupancy query that picks the cluster form runs during the capture;
+    # at 1M tokens the 16-CTA opt-in is not set there, and the portable size runs
     import os
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    out = subprocess.run([sys.executable, "-c", CAPTURE_FIRST, root], capture_output=True,
-                         text=True, timeout=300)
+    out = subprocess.run([sys.executable, "-c", CAPTURE_FIRST, root, str(length)],
+                         capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     assert out.stdout.strip().endswith("ok")
 

@@ -9,8 +9,9 @@
 //
 // Work split: two kernels.
 //   1. canvas_origin_kernel, one CTA per prompt chunk (or, for long chunks, a
-//      cluster of K CTAs that deal the blocks of ids round-robin and exchange
-//      their minima through distributed shared memory after each round),
+//      cluster of K <= 16 CTAs that deal the blocks of ids round-robin and
+//      exchange their minima through distributed shared memory after each
+//      round),
 //      finds the chunk's first marker (16 loads in flight per thread, warp
 //      `redux.sync` min, a shared-memory min) and stops at the first block
 //      (round) of ids that holds one, so no id is read twice; it writes the
@@ -44,7 +45,8 @@ constexpr int kPosThreads = 512;
 constexpr int kSliceTarget = 2048;                          // tokens per planes CTA
 constexpr int kMaxSlices = 65535;                           // gridDim.y limit
 constexpr int kQwenVlFrameShift = kGridRows + 1;            // start = O + 65
-constexpr int kOriginMaxCluster = 8;                        // CTAs per long chunk
+constexpr int kOriginMaxCluster = 16;                       // CTAs per long chunk
+constexpr int kPortableCluster = 8;                         // above: opt-in per kernel
 
 // The ids of the block seq[c, c + kScanChunk) this thread reads (16 loads in
 // flight), entries past len reading as a non-marker.
@@ -262,6 +264,35 @@ __global__ void canvas_positions_step_kernel(const int32_t* __restrict__ cache_l
   }
 }
 
+// Whether clusters of more than kPortableCluster origin CTAs are enabled on the
+// current device: the opt-in is a function attribute, set once per device
+// and never while `stream` is being captured (that call then keeps to the
+// portable size).
+bool origin_large_clusters(cudaStream_t stream) {
+  static std::mutex mu;
+  static bool enabled[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return false;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (enabled[dev]) return true;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (cap != cudaStreamCaptureStatusNone) return false;
+  if (cudaFuncSetAttribute(canvas_origin_kernel<true>,
+                           cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  enabled[dev] = true;
+  return true;
+}
+
 // Whether the current device can hold at least one cluster of k origin CTAs
 // (occupancy query, no launch; cached per device and k).
 bool origin_clusters_fit(int k, const cudaLaunchConfig_t& cfg) {
@@ -302,6 +333,7 @@ cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlen
   const int64_t avg = (n_tokens + num_seqs - 1) / num_seqs;
   int k = 1;
   while (k < kOriginMaxCluster && static_cast<int64_t>(k) * 4 * kScanChunk < avg) k *= 2;
+  if (k > kPortableCluster && !origin_large_clusters(stream)) k = kPortableCluster;
   if (k == 1) {
     canvas_origin_kernel<false><<<static_cast<unsigned>(num_seqs), kOriginThreads, 0, stream>>>(
         ids, cu_seqlens, num_seqs, n_tokens, image_token_id, rule, pos_offset, in_start,
