@@ -328,11 +328,21 @@ cudaError_t launch_positions_origin(const int32_t* ids, const int32_t* cu_seqlen
                                    int32_t* out_start, int32_t* out_amount,
                                    int32_t* device_status, cudaStream_t stream) {
   if (num_seqs == 0) return cudaSuccess;
-  // Chunks averaging more than four blocks of ids get a cluster of K CTAs
-  // (K a power of two up to kOriginMaxCluster, one per four blocks).
+  // Chunks averaging more than two blocks of ids get a cluster of K CTAs: K a
+  // power of two up to kOriginMaxCluster, one CTA per two blocks, and no
+  // more CTAs in all than the SMs (each cluster CTA fills an SM), so that
+  // every cluster runs in the first wave.
   const int64_t avg = (n_tokens + num_seqs - 1) / num_seqs;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
   int k = 1;
-  while (k < kOriginMaxCluster && static_cast<int64_t>(k) * 4 * kScanChunk < avg) k *= 2;
+  while (k < kOriginMaxCluster && static_cast<int64_t>(k) * 2 * kScanChunk < avg &&
+         static_cast<int64_t>(num_seqs) * 2 * k <= 2 * static_cast<int64_t>(sms))
+    k *= 2;
   if (k > kPortableCluster && !origin_large_clusters(stream)) k = kPortableCluster;
   if (k == 1) {
     canvas_origin_kernel<false><<<static_cast<unsigned>(num_seqs), kOriginThreads, 0, stream>>>(
