@@ -95,53 +95,54 @@ __device__ __forceinline__ int64_t first_marker(const int32_t* __restrict__ seq,
 }
 
 // first_marker by the K CTAs of this CTA's cluster: in round i, rank r scans
-// block i * K + r; after each round lane q < K of warp 0 reads rank q's
-// minimum through distributed shared memory (double-buffered, so one cluster
-// barrier per round suffices), and the CTA's threads read the cluster's
-// minimum from warp 0; all stop at the first round that found a marker.
-// Each rank's loads for the next round are issued before that exchange, so
-// their latency overlaps it; no id is read twice, and at most one round past
-// the first marker is read.  Cluster-uniform result; every thread of every
-// CTA of the cluster must call it.  Local indices fit in int32 (a chunk's
-// length comes from int32 cu_seqlens).
+// block i * K + r; each warp's minimum goes straight into the leader CTA's
+// slot for the round (an atomicMin in its shared memory, through distributed
+// shared memory), one cluster barrier ends the round, and lane 0 of every
+// warp reads the slot back for its warp; all stop at the first round that
+// found a marker.  Three slots rotate: the leader resets the slot of round
+// i + 2 after round i's barrier, when every CTA has read it (in round i - 1)
+// and none can write it before round i + 1's barrier.  Each rank's loads for
+// the next round are issued before the exchange; no id is read twice, and
+// at most one round past the first marker is read.  Cluster-uniform result;
+// every thread of every CTA of the cluster must call it.  Local indices fit
+// in int32 (a chunk's length comes from int32 cu_seqlens).
 __device__ __forceinline__ int64_t first_marker_cluster(const int32_t* __restrict__ seq,
                                                         int64_t len, int32_t marker,
-                                                        int* s_warp_min, int* s_found,
-                                                        int* s_all) {
+                                                        int* s_slots) {
   cg::cluster_group cluster = cg::this_cluster();
   const int64_t K = cluster.num_blocks();
   const int64_t r = cluster.block_rank();
+  const int lane = threadIdx.x & 31;
   const int64_t blocks = (len + kScanChunk - 1) / kScanChunk;
+  int* const leader = cluster.map_shared_rank(s_slots, 0);
+  if (threadIdx.x < 3) s_slots[threadIdx.x] = INT_MAX;
+  cluster.sync();  // the leader's slots are set before any rank writes them
   int64_t result = -1;
   int32_t v[kIdsPerThread];
   load_block(seq, r * kScanChunk, len, marker, v);
   for (int64_t i = 0; i * K < blocks; ++i) {
     const int64_t c = (i * K + r) * kScanChunk;
-    int mine = INT_MAX;
+    int best = INT_MAX;
     if (c < len) {
-      const int best = block_min(v, marker, s_warp_min);
-      if (best != INT_MAX) mine = static_cast<int>(c + best);
+#pragma unroll
+      for (int m = kIdsPerThread - 1; m >= 0; --m)
+        if (v[m] == marker) best = static_cast<int>(c) + m * kOriginThreads + threadIdx.x;
     }
+    best = __reduce_min_sync(0xffffffffu, best);
     if ((i + 1) * K < blocks) load_block(seq, c + K * kScanChunk, len, marker, v);
-    int* const slot = s_found + (i & 1);
-    if (threadIdx.x == 0) *slot = mine;
+    const int slot = static_cast<int>(i % 3);
+    if (lane == 0 && best != INT_MAX) atomicMin(leader + slot, best);
     cluster.sync();
-    if (threadIdx.x < 32) {
-      const int q = threadIdx.x;
-      const int m = q < K ? *cluster.map_shared_rank(slot, q) : INT_MAX;
-      const int all = __reduce_min_sync(0xffffffffu, m);
-      if (q == 0) *s_all = all;
-    }
-    __syncthreads();
-    // warp 0 rewrites s_all only after the next round's cluster barrier, which
-    // every thread of the CTA reaches after this read
-    const int all = *s_all;
+    if (r == 0 && threadIdx.x == 0) s_slots[(i + 2) % 3] = INT_MAX;
+    int all = 0;
+    if (lane == 0) all = leader[slot];
+    all = __shfl_sync(0xffffffffu, all, 0);
     if (all != INT_MAX) {
       result = all;
       break;
     }
   }
-  cluster.sync();  // no CTA leaves while a peer may still read its s_found
+  cluster.sync();  // no CTA leaves while a peer may still read or write its slots
   return result;
 }
 
@@ -171,8 +172,7 @@ __global__ void __launch_bounds__(kOriginThreads)
                          const int32_t* __restrict__ in_amount, int32_t* __restrict__ out_start,
                          int32_t* __restrict__ out_amount, int32_t* __restrict__ status) {
   __shared__ int s_warp_min[kOriginThreads / 32];
-  __shared__ int s_found[2];
-  __shared__ int s_all;
+  __shared__ int s_slots[3];
   pdl::launch_dependents();
   // the chunk of this CTA (of its cluster), and whether it writes the results
   int32_t b = blockIdx.x;
@@ -196,8 +196,7 @@ __global__ void __launch_bounds__(kOriginThreads)
     start = kTextOnlyStart;
     amount = 0;
   } else if (start >= kTextOnlyStart) {
-    const int64_t m = kCluster ? first_marker_cluster(ids + first, len, marker, s_warp_min, s_found,
-                                                    &s_all)
+    const int64_t m = kCluster ? first_marker_cluster(ids + first, len, marker, s_slots)
                                : first_marker(ids + first, len, marker, s_warp_min);
     if (m >= 0) {
       const int64_t origin = (pos_offset ? __ldg(pos_offset + b) : 0) + m;
