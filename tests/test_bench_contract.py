@@ -45,6 +45,12 @@ def test_source_hash_ignores_comments_but_not_code():
     assert bench.code_tokens('f("a//b"); // c') == 'f("a//b");'
 
 
+def test_host_cpu_record():
+    h = bench.host_cpu()
+    assert h["nproc"] == os.cpu_count() and h["threads_allowed"] == bench.host_cores()
+    assert h["cpu_model"] is None or isinstance(h["cpu_model"], str)
+
+
 def test_oracle_sample_step_threads_agree():
     wl = inputs.make_config(2)
     wl_cpu = bench.cpu_sample_inputs(wl, 600)
@@ -64,6 +70,8 @@ def test_reference_arm_prints_one_json_line():
     assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    host = d["cpu_baseline"]["host"]
+    assert host["nproc"] >= 1 and host["threads_allowed"] >= 1 and "cpu_model" in host
     # the same config keys (and workload) as the GPU arm's line
     assert set(d["config"]) == {"workload", "global_batch", "launch", "op", "step", "seq_len",
                                 "parallelism", "l2"}
