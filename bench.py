@@ -13,6 +13,9 @@ instead, and times the rotate launch on its own.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...   (weak scaling: one batch per GPU)
     python bench.py --probe copy-pattern   (the staged copy-pattern ceiling alone)
+    python bench.py --op frames            (multi-frame planes, 256 x 65,536 tokens)
+    python bench.py --op chunk [--chunks C] [--rule canvas|qwen_vl|planes_1d]
+                                           (chunked prefill planes on the same prompts)
 
 Prints one JSON line on rank 0.  --impl reference times the fp64 CPU oracle on
 all host cores (a thread pool over token ranges) on a bounded sample of the
@@ -42,6 +45,7 @@ METRIC = "canvas M-RoPE tokens/s and achieved HBM GB/s (% of B200 peak), bf16 Q/
 UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e specification (DGX figure)
+PLANES_OPS = ("frames", "chunk")  # planes-only steps on 65,536-token prompts
 ROTATE_SOURCES = ["vlm_decoder_positional_b200/csrc/rotate.cu",
                   "vlm_decoder_positional_b200/csrc/rotate_staged.cu",
                   "vlm_decoder_positional_b200/csrc/tma.cuh",
@@ -707,26 +711,112 @@ def run_probe_only(args):
     return 0
 
 
-def frames_config(args, wl, world):
+def chunk_bytes(n_tokens, num_seqs, chunks, id_reads):
+    """Chunked prefill planes, one cmr_positions_chunk call per chunk: 12 B of
+    planes per token; the ids the rule has to read (``id_reads`` in all, see
+    first_marker_reads), 4 B each; per prompt and call cu_seqlens and the
+    outgoing state (12 B), and from the second chunk on the offset and the
+    incoming state (12 B more).  The planes themselves follow from each
+    token's absolute index and the state, so no other id is needed."""
+    return n_tokens * 12 + id_reads * 4 + num_seqs * (12 * chunks + 12 * (chunks - 1))
+
+
+def first_marker_reads(ids, cu_seqlens, marker, rule):
+    """Ids a rule must read to fix every prompt's state: up to and including
+    the prompt's first marker, or all of it when it holds none (canvas and
+    Qwen-VL rules); none under planes_1d, which never shifts."""
+    if rule == "planes_1d":
+        return 0
+    total = 0
+    for b in range(cu_seqlens.shape[0] - 1):
+        seg = ids[cu_seqlens[b]:cu_seqlens[b + 1]]
+        hit = np.flatnonzero(seg == marker)
+        total += int(hit[0]) + 1 if hit.size else int(seg.shape[0])
+    return total
+
+
+def planes_workload(args, seed=None):
+    """The planes-only workloads: --op frames, prompts of 65,536 tokens with
+    --frames-per-prompt frames on a --grid-side grid; --op chunk, the same
+    prompts with one thumbnail each (grid side 8) at a random origin."""
+    if args.op == "frames":
+        return inputs.make_frames_workload(num_prompts=args.prompts,
+                                           frames=args.frames_per_prompt,
+                                           grid_side=args.grid_side, seed=seed)
+    return inputs.make_frames_workload(num_prompts=args.prompts, frames=1, grid_side=8,
+                                       seed=seed)
+
+
+def chunk_pieces(ids, cu_seqlens, chunks):
+    """Cuts every prompt of an equal-length batch into ``chunks`` equal pieces:
+    piece c of all prompts is one cmr_positions_chunk call.  Returns a list of
+    (ids, cu_seqlens, pos_offset) numpy arrays, one per call."""
+    b = cu_seqlens.shape[0] - 1
+    length = int(cu_seqlens[1] - cu_seqlens[0]) if b else 0
+    if b == 0 or not np.array_equal(cu_seqlens, np.arange(b + 1, dtype=np.int64) * length):
+        raise ValueError("chunked prefill needs prompts of one length")
+    if chunks < 1 or length % chunks:
+        raise ValueError(f"{chunks} chunks do not divide prompts of {length} tokens")
+    lc = length // chunks
+    blocks = np.asarray(ids, np.int32).reshape(b, chunks, lc)
+    cu = (np.arange(b + 1) * lc).astype(np.int32)
+    return [(np.ascontiguousarray(blocks[:, c, :]).reshape(-1), cu,
+             np.full(b, c * lc, np.int32)) for c in range(chunks)]
+
+
+def oracle_planes_work(args, wl):
+    """The oracle's planes of the first ``take`` prompts of a planes workload:
+    run(take) -> tokens covered (the frames reading, or the chunked prefill
+    carrying each prompt's state from chunk to chunk)."""
+    import oracle
+    cu = wl.cu_seqlens
+    if args.op == "frames":
+        def run(lo, hi):
+            oracle.positions_frames(wl.ids[cu[lo]:cu[hi]], cu[lo:hi + 1] - cu[lo],
+                                    wl.image_token_id, args.grid_side)
+            return int(cu[hi] - cu[lo])
+        return run
+
+    def run(lo, hi):
+        pieces = chunk_pieces(wl.ids[cu[lo]:cu[hi]], cu[lo:hi + 1] - cu[lo], args.chunks)
+        state = (None, None)
+        for ids_c, cu_c, off_c in pieces:
+            _, st, am = oracle.positions_chunk(ids_c, cu_c, wl.image_token_id, args.rule,
+                                               off_c, *state)
+            state = (st, am)
+        return int(cu[hi] - cu[lo])
+    return run
+
+
+def planes_config(args, wl, world):
     n, b = wl.n_tokens, wl.num_seqs
-    return {"workload": f"{wl.name}: {b} prompts x {n // b} tokens, "
-                        f"{args.frames_per_prompt} frames each, grid side {args.grid_side}",
-            "global_batch": n * world, "launch": args.launch, "op": "frames",
-            "step": "separate", "seq_len": n // b,
+    if args.op == "frames":
+        what = (f"{wl.name}: {b} prompts x {n // b} tokens, "
+                f"{args.frames_per_prompt} frames each, grid side {args.grid_side}")
+        moved = positions_bytes(n, b)
+    else:
+        what = (f"chunked_prefill_{b}x{n // b}: {b} prompts x {n // b} tokens, one 448x448 "
+                f"thumbnail each, {args.chunks} chunks per prompt, rule {args.rule}")
+        moved = chunk_bytes(n, b, args.chunks, first_marker_reads(
+            wl.ids, wl.cu_seqlens, wl.image_token_id, args.rule))
+    return {"workload": what, "global_batch": n * world, "launch": args.launch, "op": args.op,
+            "step": "separate" if args.op == "frames" else f"{args.chunks} chunk calls",
+            "seq_len": n // b,
             "parallelism": f"dp{world} (independent batches, no data-path collective)",
             "l2": "inputs larger than L2 (%.0f MB of ids and planes per step, L2 126 MB); no "
-                  "flush" % (positions_bytes(n, b) / 1e6)}
+                  "flush" % (moved / 1e6) if moved > 126e6 else
+                  "ids and planes (%.0f MB) fit in L2; no flush" % (moved / 1e6)}
 
 
-def run_frames_reference(args):
-    """--impl reference --op frames: the oracle's multi-frame planes on all
-    host cores (whole prompts split over a thread pool), on a bounded sample
-    of the multi-frame workload per step."""
+def run_planes_reference(args):
+    """--impl reference --op frames|chunk: the oracle's planes on all host
+    cores (whole prompts split over a thread pool), on a bounded sample of the
+    workload per step."""
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    import oracle
     from concurrent.futures import ThreadPoolExecutor
-    wl = inputs.make_frames_workload(frames=args.frames_per_prompt, grid_side=args.grid_side)
+    wl = planes_workload(args)
+    work = oracle_planes_work(args, wl)
     cores = host_cores()
     cu = wl.cu_seqlens
 
@@ -734,10 +824,8 @@ def run_frames_reference(args):
         cuts = np.linspace(0, take, cores + 1).astype(int)
 
         def part(i):
-            lo, hi = cuts[i], cuts[i + 1]
-            if hi > lo:
-                oracle.positions_frames(wl.ids[cu[lo]:cu[hi]], cu[lo:hi + 1] - cu[lo],
-                                        wl.image_token_id, args.grid_side)
+            if cuts[i + 1] > cuts[i]:
+                work(cuts[i], cuts[i + 1])
         with ThreadPoolExecutor(cores) as ex:
             list(ex.map(part, range(cores)))
 
@@ -757,14 +845,16 @@ def run_frames_reference(args):
     dt = time.perf_counter() - t0
     n = int(cu[take])
     value = n * args.steps / dt
-    sample = (f"per step: multi-frame planes of the first {take} prompts ({n} tokens), "
+    what = ("multi-frame planes" if args.op == "frames" else
+            f"planes in {args.chunks} chunks per prompt (rule {args.rule})")
+    sample = (f"per step: {what} of the first {take} prompts ({n} tokens), "
               f"the oracle (integer arithmetic) on {cores} host threads")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int32", "data": "synthetic (seeded)",
-        "config": frames_config(args, wl, args.gpus),
+        "config": planes_config(args, wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample, "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -773,10 +863,13 @@ def run_frames_reference(args):
     return 0
 
 
-def run_frames(args):
+def run_planes(args):
     """--op frames: one step = cmr_positions_frames (multi-frame canvas planes)
-    on the multi-frame workload (256 prompts x 65,536 tokens, 32 frames each,
-    grid side --grid-side), graph-replayed, CUDA events around each call."""
+    on 65,536-token prompts with --frames-per-prompt frames on a --grid-side
+    grid.  --op chunk: one step = the chunked prefill of every prompt, --chunks
+    cmr_positions_chunk calls (chunk c of all prompts per call, each carrying
+    the state of the call before it) under --rule.  Graph-replayed, CUDA events
+    around the K steps."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -788,19 +881,41 @@ def run_frames(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     cmr.lib()
     seed = shard.rank_seed(inputs.BASE_SEED + 6, rank)
-    wl = inputs.make_frames_workload(frames=args.frames_per_prompt, grid_side=args.grid_side,
-                                     seed=seed)
+    wl = planes_workload(args, seed=seed)
     n, b = wl.n_tokens, wl.num_seqs
-    ids = torch.from_numpy(wl.ids).to(dev)
-    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
-    pos = torch.empty((3, n), dtype=torch.int32, device=dev)
-    start = torch.empty(b, dtype=torch.int32, device=dev)
-    amount = torch.empty(b, dtype=torch.int32, device=dev)
-    ws = torch.empty(cmr.positions_frames_workspace_bytes(b, n), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if args.op == "frames":
+        ids = torch.from_numpy(wl.ids).to(dev)
+        cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+        pos = torch.empty((3, n), dtype=torch.int32, device=dev)
+        start = torch.empty(b, dtype=torch.int32, device=dev)
+        amount = torch.empty(b, dtype=torch.int32, device=dev)
+        ws = torch.empty(cmr.positions_frames_workspace_bytes(b, n), dtype=torch.uint8,
+                         device=dev)
 
-    def call():
-        cmr.positions_frames(ids, cu, args.grid_side, out=(pos, start, amount), workspace=ws)
+        def call():
+            cmr.positions_frames(ids, cu, args.grid_side, out=(pos, start, amount),
+                                 workspace=ws)
+        moved, launches = positions_bytes(n, b), 2
+        kernel = "frames_positions_kernel (+ frames_summary_kernel)"
+        timed = "the summary and planes kernels"
+    else:
+        pieces = [tuple(torch.from_numpy(a).to(dev) for a in p)
+                  for p in chunk_pieces(wl.ids, wl.cu_seqlens, args.chunks)]
+        outs = [torch.empty((3, p[0].numel()), dtype=torch.int32, device=dev) for p in pieces]
+        states = [(torch.empty(b, dtype=torch.int32, device=dev),
+                   torch.empty(b, dtype=torch.int32, device=dev)) for _ in range(2)]
+
+        def call():
+            for c, (ids_c, cu_c, off_c) in enumerate(pieces):
+                cmr.positions_chunk(ids_c, cu_c, pos_offset=off_c if c else None,
+                                    state=states[(c + 1) % 2] if c else None, rule=args.rule,
+                                    out=(outs[c], *states[c % 2]))
+        moved = chunk_bytes(n, b, args.chunks, first_marker_reads(
+            wl.ids, wl.cu_seqlens, wl.image_token_id, args.rule))
+        launches = 2 * args.chunks
+        kernel = "canvas_positions_kernel (+ canvas_origin_kernel), per chunk"
+        timed = f"the {args.chunks} chunk calls (origin scan and planes kernels each)"
 
     call()
     torch.cuda.synchronize(dev)
@@ -827,29 +942,28 @@ def run_frames(args):
         dist.barrier()
     ms_local = t_begin.elapsed_time(t_end)
     ms_max = shard.max_over_ranks(ms_local, dist, dev)
-    call_ms = ms_local / args.steps
-    moved = positions_bytes(n, b)
+    step_ms = ms_local / args.steps
     if rank == 0:
         peak, peak_src = measured_peak()
-        achieved = moved / (call_ms / 1e3) / 1e9
+        achieved = moved / (step_ms / 1e3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            cores = 1
+            work = oracle_planes_work(args, wl)
             take = 1
             t0 = time.perf_counter()
             while True:  # whole prompts, about --cpu-seconds of oracle work
-                oracle.positions_frames(wl.ids[: wl.cu_seqlens[take]], wl.cu_seqlens[: take + 1],
-                                        wl.image_token_id, args.grid_side)
+                tokens = work(0, take)
                 dt = time.perf_counter() - t0
                 if dt > args.cpu_seconds or take == b:
                     break
                 take = min(b, take * 2)
                 t0 = time.perf_counter()
-            cpu = {"value": int(wl.cu_seqlens[take]) / dt, "unit": UNIT, "cores": cores,
-                   "kind": "oracle", "host": host_cpu(),
-                   "sample": f"multi-frame planes of the first {take} prompts "
-                             f"({int(wl.cu_seqlens[take])} tokens), 1 thread, {dt:.2f} s"}
+            what = ("multi-frame planes" if args.op == "frames" else
+                    f"planes in {args.chunks} chunks per prompt (rule {args.rule})")
+            cpu = {"value": tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "host": host_cpu(),
+                   "sample": f"{what} of the first {take} prompts ({tokens} tokens), "
+                             f"1 thread, {dt:.2f} s"}
         tokens_all = n * world
         out = {
             "metric": METRIC, "value": tokens_all * args.steps / (ms_max / 1e3), "unit": UNIT,
@@ -857,19 +971,18 @@ def run_frames(args):
             "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int32",
             "data": "synthetic (seeded uniform text ids, frames on a grid_side x grid_side grid)",
-            "config": frames_config(args, wl, world),
+            "config": planes_config(args, wl, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
-                         "kernel": "frames_positions_kernel (+ frames_summary_kernel)",
-                         "algorithmic_bytes_per_launch": moved, "avg_launch_ms": call_ms,
-                         "timed": "the call (CUDA events around the K calls, divided by K): "
-                                  "the summary and planes kernels",
+                         "frac": achieved / peak, "traffic": None, "kernel": kernel,
+                         "algorithmic_bytes_per_launch": moved, "avg_launch_ms": step_ms,
+                         "timed": f"the step (CUDA events around the K steps, divided by K): "
+                                  f"{timed}",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6650 GB/s",
                          "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS},
-            "e2e": {"skipped": "--op frames times the device step only"},
-            "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "cpu_baseline": cpu,
-            "impl": "ours",
+            "e2e": {"skipped": f"--op {args.op} times the device step only"},
+            "gpu_launches": launches * args.steps, "clocks": clocks.summary(),
+            "cpu_baseline": cpu, "impl": "ours",
         }
         print(json.dumps(out), flush=True)
     if dist:
@@ -991,10 +1104,18 @@ def main():
     ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
                     help="weak: a full batch per GPU (default); strong: one batch split by "
                          "whole prompts")
-    ap.add_argument("--op", choices=["rotate", "shift", "cache", "frames"], default="rotate",
+    ap.add_argument("--op", choices=["rotate", "shift", "cache", *PLANES_OPS], default="rotate",
                     help="rotate: planes from pos (default); shift: planes derived in the "
                          "rotate kernel; cache: rotate + KV-cache write; frames: the "
-                         "multi-frame planes alone on their own workload")
+                         "multi-frame planes alone on their own workload; chunk: the planes "
+                         "of a chunked prefill (cmr_positions_chunk) on that workload's "
+                         "prompts with one thumbnail each")
+    ap.add_argument("--prompts", type=int, default=256,
+                    help="--op frames|chunk: prompts of 65,536 tokens in the batch")
+    ap.add_argument("--chunks", type=int, default=4,
+                    help="--op chunk: equal chunks per prompt, one call each")
+    ap.add_argument("--rule", choices=sorted(cmr.RULES), default="canvas",
+                    help="--op chunk: the position rule of cmr_positions_chunk")
     ap.add_argument("--grid-side", type=int, default=8,
                     help="--op frames: side of each frame's grid (8: 448x448 thumbnail)")
     ap.add_argument("--frames-per-prompt", type=int, default=32,
@@ -1020,11 +1141,11 @@ def main():
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
-        return run_frames_reference(args) if args.op == "frames" else run_reference(args)
+        return run_planes_reference(args) if args.op in PLANES_OPS else run_reference(args)
     if args.probe:
         return run_probe_only(args)
-    if args.op == "frames":
-        return run_frames(args)
+    if args.op in PLANES_OPS:
+        return run_planes(args)
     return run_ours(args)
 
 

@@ -7,6 +7,8 @@ import sys
 
 import pytest
 
+import bench
+
 pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -59,3 +61,50 @@ def test_separate_step_and_the_copy_pattern_probe():
     assert d["positions_avg_ms"] > 0
     d = run_bench("--probe", "copy-pattern", "--workload", "2", "--steps", "5", "--warmup", "3")
     assert d["probe"] == "copy-pattern" and d["gbs"] > 0 and d["launches"] == 5
+
+
+@pytest.mark.parametrize("op", ["frames", "chunk"])
+def test_planes_ops(op):
+    d = run_bench("--op", op, "--prompts", "16", "--rule", "qwen_vl", "--steps", "4",
+                  "--warmup", "3", "--cpu-seconds", "1")
+    assert d["value"] > 0 and d["config"]["op"] == op and d["config"]["global_batch"] == 16 * 65536
+    assert d["gpu_launches"] == (2 if op == "frames" else 2 * 4) * 4
+    r = d["roofline"]
+    assert r["bound"] == "hbm" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
+    assert "skipped" in d["e2e"] and d["cpu_baseline"]["kind"] == "oracle"
+    if op == "chunk":
+        # planes, the ids up to each prompt's first marker (one thumbnail each), the state
+        n = 16 * 65536
+        assert bench.chunk_bytes(n, 16, 4, 16) < r["algorithmic_bytes_per_launch"]
+        assert r["algorithmic_bytes_per_launch"] < bench.chunk_bytes(n, 16, 4, n)
+
+
+@pytest.mark.parametrize("rule", ["canvas", "qwen_vl", "planes_1d"])
+def test_the_chunk_step_equals_the_oracle(cuda_device, rule):
+    # the chunk op's calls as bench.py makes them (no offset or state for the
+    # first chunk, two state buffers in turn): every plane and the state after
+    # each chunk equal the oracle's, bit for bit
+    import numpy as np
+    import torch
+
+    import oracle
+    from vlm_decoder_positional_b200 import cmr, inputs
+    dev = cuda_device
+    wl = inputs.make_frames_workload(num_prompts=16, frames=1, seed=77)
+    pieces = bench.chunk_pieces(wl.ids, wl.cu_seqlens, 8)
+    states = [(torch.empty(16, dtype=torch.int32, device=dev),
+               torch.empty(16, dtype=torch.int32, device=dev)) for _ in range(2)]
+    o_state = (None, None)
+    for c, (ids_c, cu_c, off_c) in enumerate(pieces):
+        g = [torch.from_numpy(a).to(dev) for a in (ids_c, cu_c, off_c)]
+        pos = torch.empty((3, ids_c.shape[0]), dtype=torch.int32, device=dev)
+        cmr.positions_chunk(g[0], g[1], pos_offset=g[2] if c else None,
+                            state=states[(c + 1) % 2] if c else None, rule=rule,
+                            out=(pos, *states[c % 2]))
+        torch.cuda.synchronize()
+        want, ws, wa = oracle.positions_chunk(ids_c, cu_c, wl.image_token_id, rule, off_c,
+                                              *o_state)
+        np.testing.assert_array_equal(pos.cpu().numpy(), want)
+        np.testing.assert_array_equal(states[c % 2][0].cpu().numpy(), ws)
+        np.testing.assert_array_equal(states[c % 2][1].cpu().numpy(), wa)
+        o_state = (ws, wa)
