@@ -685,6 +685,30 @@ def run_plain_copy_probe(moved, dev, stream, launches=10, warmup=3):
                     "contiguous buffers); mean of %d copies" % launches}
 
 
+def run_plain_fill_probe(nbytes, dev, stream, launches=10, warmup=3):
+    """A store-only stream (torch fill_) of ``nbytes``, timed the same way as
+    the copy probe: the ceiling of a launch that only writes, as the planes
+    kernels mostly do."""
+    buf = torch.empty((nbytes + 15) // 16 * 4, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            buf.fill_(7)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(launches)]
+        torch.cuda.synchronize(dev)
+        for a, z in ev:
+            a.record(stream)
+            buf.fill_(7)
+            z.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(z) for a, z in ev)
+    size = buf.numel() * 4
+    del buf
+    return {"gbs": size / (ms / 1e3) / 1e9, "ms": ms, "bytes": size,
+            "what": "torch fill_ of a buffer the size of the planes (stores only); mean of "
+                    "%d fills" % launches}
+
+
 def run_probe_only(args):
     """--probe copy-pattern: the ceiling probe alone on the workload's Q/K."""
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
@@ -946,6 +970,9 @@ def run_planes(args):
     if rank == 0:
         peak, peak_src = measured_peak()
         achieved = moved / (step_ms / 1e3) / 1e9
+        # the planes' stores against a store-only stream of the same size
+        fill = run_plain_fill_probe(12 * n, dev, stream)
+        planes_gbs = 12 * n / (step_ms / 1e3) / 1e9
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             work = oracle_planes_work(args, wl)
@@ -979,7 +1006,10 @@ def run_planes(args):
                                   f"{timed}",
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_src == "measured" else "fallback 6650 GB/s",
-                         "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS},
+                         "spec_peak": SPEC_HBM_GBS, "frac_of_spec": achieved / SPEC_HBM_GBS,
+                         "planes_store_gbs": planes_gbs, "same_size_fill_gbs": fill["gbs"],
+                         "planes_frac_of_fill": planes_gbs / fill["gbs"],
+                         "same_size_fill_what": fill["what"]},
             "e2e": {"skipped": f"--op {args.op} times the device step only"},
             "gpu_launches": launches * args.steps, "clocks": clocks.summary(),
             "cpu_baseline": cpu, "impl": "ours",

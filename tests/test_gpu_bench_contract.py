@@ -72,6 +72,8 @@ def test_planes_ops(op):
     r = d["roofline"]
     assert r["bound"] == "hbm" and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
     assert "skipped" in d["e2e"] and d["cpu_baseline"]["kind"] == "oracle"
+    assert r["same_size_fill_gbs"] > 0 and r["planes_store_gbs"] > 0
+    assert abs(r["planes_frac_of_fill"] - r["planes_store_gbs"] / r["same_size_fill_gbs"]) < 1e-9
     if op == "chunk":
         # planes, the ids up to each prompt's first marker (one thumbnail each), the state
         n = 16 * 65536
