@@ -98,9 +98,9 @@ typedef enum cmr_status {
  *                The library never clears it.
  * Two kernels: one CTA per prompt (a cluster of up to 16 CTAs when prompts
  * average more than 65,536 tokens) scans its ids up to the first marker (no
- * id is read twice) and writes the state; then CTAs over slices of about
- * 2,048 tokens write the planes, reading the state back from out_start /
- * out_amount.
+ * id is read twice) and writes the state; then CTAs over slices of 2,048
+ * tokens (8,192 where the batch still fills three waves of CTAs) write the
+ * planes, reading the state back from out_start / out_amount.
  * Errors: CMR_EINVAL for null required pointers, negative sizes, num_seqs = 0
  * with n_tokens > 0, or n_tokens > INT32_MAX. */
 CMR_API cmr_status cmr_positions(const int32_t* ids, const int32_t* cu_seqlens,

@@ -17,7 +17,7 @@
 //      (round) of ids that holds one, so no id is read twice; it writes the
 //      chunk's outgoing state (start, amount) -- carried over when a frame is
 //      already known, (2^30, 0) for text and for the 1-D rule.
-//   2. canvas_positions_kernel, CTAs (b, s) over slices of about 2,048 tokens,
+//   2. canvas_positions_kernel, CTAs (b, s) over slices of 2,048 to 8,192 tokens,
 //      launched programmatically behind the first (it starts while the scan
 //      runs and waits for it before reading the state), writes the planes:
 //      12 B per token, no ids read.
@@ -42,7 +42,8 @@ constexpr int kOriginThreads = 1024;
 constexpr int kIdsPerThread = 16;
 constexpr int kScanChunk = kOriginThreads * kIdsPerThread;  // 16,384 ids per step
 constexpr int kPosThreads = 512;
-constexpr int kSliceTarget = 2048;                          // tokens per planes CTA
+constexpr int kSliceMin = 2048;                             // tokens per planes CTA, and
+constexpr int kSliceMax = 8192;                             //   for batches of many waves
 constexpr int kMaxSlices = 65535;                           // gridDim.y limit
 constexpr int kQwenVlFrameShift = kGridRows + 1;            // start = O + 65
 constexpr int kOriginMaxCluster = 16;                       // CTAs per long chunk
@@ -383,8 +384,22 @@ cudaError_t launch_positions(const int32_t* ids, const int32_t* cu_seqlens, int3
                                           rule, pos_offset, in_start, in_amount, out_start,
                                           out_amount, device_status, stream);
   if (e != cudaSuccess || n_tokens == 0) return e;
+  // Slices of kSliceMin tokens, or of kSliceMax where even those leave at
+  // least three resident waves of CTAs: each CTA's start (the bounds, the
+  // programmatic wait, the state) is two dependent memory round trips, which
+  // long slices spread over more stores, while a grid of one or two waves
+  // loses more to its partly filled last wave than it saves.
   const int64_t avg = (n_tokens + num_seqs - 1) / num_seqs;
-  int64_t slices = (avg + kSliceTarget - 1) / kSliceTarget;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const int64_t wave = static_cast<int64_t>(sms) * (2048 / kPosThreads);
+  int64_t slices = (avg + kSliceMax - 1) / kSliceMax;
+  if (static_cast<int64_t>(num_seqs) * slices < 3 * wave)
+    slices = (avg + kSliceMin - 1) / kSliceMin;
   slices = slices < 1 ? 1 : (slices > kMaxSlices ? kMaxSlices : slices);
   const dim3 grid(static_cast<unsigned>(num_seqs), static_cast<unsigned>(slices));
   return pdl::launch(canvas_positions_kernel, grid, dim3(kPosThreads), 0, stream, true,
