@@ -824,7 +824,8 @@ def planes_config(args, wl, world):
         moved = chunk_bytes(n, b, args.chunks, first_marker_reads(
             wl.ids, wl.cu_seqlens, wl.image_token_id, args.rule))
     return {"workload": what, "global_batch": n * world, "launch": args.launch, "op": args.op,
-            "step": "separate" if args.op == "frames" else f"{args.chunks} chunk calls",
+            "step": "separate" if args.op == "frames" else
+                    f"{args.chunks} chunk call{'s' if args.chunks != 1 else ''}",
             "seq_len": n // b,
             "parallelism": f"dp{world} (independent batches, no data-path collective)",
             "l2": "inputs larger than L2 (%.0f MB of ids and planes per step, L2 126 MB); no "
