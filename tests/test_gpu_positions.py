@@ -201,6 +201,31 @@ def test_cluster_scan_first_launched_inside_a_graph_capture(cuda_device, length)
     assert out.stdout.strip().endswith("ok")
 
 
+def test_large_batch_in_long_slices(cuda_device):
+    # 256 prompts x 65,536 tokens: enough CTAs for three waves even with the
+    # planes kernel's long (8,192-token) slices.  Text-only prompts, markers
+    # on both sides of every slice edge and at the prompts' ends, and random
+    # origins; every plane bit-exact
+    rng = np.random.default_rng(1234)
+    n, F = 65536, 67
+    prompts = []
+    for i in range(256):
+        kind = i % 4
+        if kind == 0:
+            prompts.append(inputs.text_ids(rng, n))
+            continue
+        if kind == 1:
+            edge = 8192 * int(rng.integers(1, 8))
+            origin = edge - 1 if i % 8 == 1 else edge          # either side of a slice edge
+        elif kind == 2:
+            origin = n - 1 - int(rng.integers(0, F + 2))        # a frame cut off by the end
+        else:
+            origin = int(rng.integers(0, n))
+        prompts.append(inputs.prompt_ids_frames(rng, n, [origin], 8))
+    ids, cu = inputs.pack(prompts)
+    check_batch(ids, cu, cuda_device)
+
+
 def test_many_short_prompts_and_repeated_markers(cuda_device):
     rng = np.random.default_rng(4)
     lens = rng.integers(0, 90, size=5000)
