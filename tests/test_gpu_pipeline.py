@@ -8,14 +8,6 @@ from vlm_decoder_positional_b200 import cmr, inputs, pipeline
 pytestmark = pytest.mark.gpu
 
 
-def test_prompt_chunks_cover_the_batch():
-    cu = np.array([0, 5, 5, 30, 31, 100, 101], np.int64)
-    ch = pipeline.prompt_chunks(cu, 30)
-    assert ch[0][0] == 0 and ch[-1][1] == 6
-    assert all(a[1] == b[0] for a, b in zip(ch, ch[1:]))
-    assert all(cu[s1] - cu[s0] <= 30 or s1 - s0 == 1 for s0, s1 in ch)
-
-
 @pytest.mark.parametrize("cfg,chunk", [(2, 1000), (3, 3 * 4096), (5, 2 * 8192)])
 def test_host_pipeline_matches_the_device_path(cuda_device, cfg, chunk):
     wl = inputs.make_config(cfg, device=cuda_device)
